@@ -1,0 +1,10 @@
+"""The CPU oracle against hand-worked values, closed forms and brute force."""
+import pytest
+
+import oracle
+import oracle_pins
+
+
+@pytest.mark.parametrize("check", oracle_pins.ALL_CHECKS, ids=lambda c: c.__name__)
+def test_oracle_pin(check):
+    check(oracle.lib())
