@@ -1,0 +1,443 @@
+"""Benchmark of the MoE expert layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Default workload: decode, T = 1 token through 40 distinct seeded layers
+(H 2048, I 512, 256 experts top-8 + 1 shared, 4-bit group 64), 18.2 GB of
+packed weights resident and cycled, so every step streams its weights from
+HBM (inputs larger than L2; no flush needed).  One step = the whole hot path
+(route, permute, expert FFN, combine) of all 40 layers, replayed as one CUDA
+graph.  A second, smaller measurement covers the T = 2048 prefill layer.
+
+Prints one JSON line on rank 0.  Under torchrun every rank runs its own
+replica (weak scaling, no collective on the data path); the time is the max
+over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+LAYERS = 40
+UNIT = "tokens/s"
+METRIC = "MoE expert-layer tokens/s (layer passes per second, T=1 decode over 40 layers)"
+
+# Algorithmic bytes of one decode layer-token (H 2048, I 512, G 64): each of
+# the 9 active experts (8 routed + shared) streams its packed gate_up and down
+# codes plus (scale, bias) pairs once; activations are 2 KB-scale.
+H, I, E, K, G = 2048, 512, 256, 8, 64
+EXPERT_BYTES = (2 * I * H + H * I) // 2 + (2 * I * (H // G) + H * (I // G)) * 4
+ROUTER_BYTES = E * H * 2
+FFN_BYTES_T1 = 9 * EXPERT_BYTES + H * 2 + H * 4      # + x (bf16) + y_acc (fp32)
+LAYER_BYTES_T1 = FFN_BYTES_T1 + ROUTER_BYTES
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=p["hbm_gbs"], bf16_tflops=p["bf16_tflops"],
+                    bf16_tflops_sustained=p.get("bf16_tflops_sustained", p["bf16_tflops"]), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+# ---------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) of SM clock and throttle reasons."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=5)
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return dict(sm_mhz=None, sm_max_mhz=mx, reasons=sorted(reasons), samples=0)
+        return dict(sm_mhz=float(np.median(sm)), sm_max_mhz=mx, reasons=sorted(reasons), samples=len(sm))
+
+
+# ------------------------------------------------------------ distributed
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def aggregate(local_ms: float, local_units: float, world: int):
+    """(max time over ranks, total units over ranks); collectives only when world > 1."""
+    if world <= 1:
+        return local_ms, local_units
+    import torch
+    import torch.distributed as dist
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" else torch.device("cpu")
+    t = torch.tensor([local_ms], dtype=torch.float64, device=dev)
+    u = torch.tensor([local_units], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------- oracle timing
+
+
+def omp_threads() -> int:
+    try:
+        import ctypes
+        return int(ctypes.CDLL("libgomp.so.1").omp_get_max_threads())
+    except OSError:
+        return os.cpu_count() or 1
+
+
+def time_oracle_decode(layers: list, budget_s: float):
+    """Layer-tokens/s of the oracle on the first layers (T = 1 each), within about budget_s."""
+    import oracle
+    done, t0 = 0, time.perf_counter()
+    while True:
+        oracle.layer(layers[done % len(layers)])
+        done += 1
+        if time.perf_counter() - t0 >= budget_s and done >= 1:
+            break
+    dt = time.perf_counter() - t0
+    return done / dt, done, dt
+
+
+# ------------------------------------------------------------- workloads
+
+
+def build_decode(device):
+    """40 seeded layers resident on the device; returns (layers, host copies of the first 3)."""
+    import gen
+    from bit_dequant_expert_b200.layer import MoELayer, to_device
+    spec = gen.config(1)
+    layers, host = [], []
+    x_all = np.empty((LAYERS, H), dtype=np.uint16)
+    for l in range(LAYERS):
+        lay = gen.make_layer(spec, l)
+        layers.append(MoELayer(lay, max_tokens=1, device=device))
+        x_all[l] = lay["x"][0]
+        if l < 3:
+            host.append(lay)
+        del lay
+    x_dev = to_device(x_all, device)
+    return layers, host, x_dev, x_all
+
+
+def _timed_replays(replay, n, stream):
+    """Device time (ms) of n calls of replay() on stream, CUDA events on that stream."""
+    import torch
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(n):
+        replay()
+    end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end)
+
+
+def _capture(fn, stream):
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    return g
+
+
+def _launch_count(layer, T):
+    import bit_dequant_expert_b200 as m
+    return m.moe_launch_count(layer.cfg, T, layer.mode, layer.path)
+
+
+def run_decode(device, steps, warmup, world, peaks):
+    import torch
+    layers, host, x_dev, x_host = build_decode(device)
+    y_dev = torch.empty(LAYERS, H, dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.Stream(device=device)
+
+    def step():
+        for l in range(LAYERS):
+            layers[l].forward(x_dev[l:l + 1], y_out=y_dev[l:l + 1])
+
+    def ffn_only():
+        for l in range(LAYERS):
+            layers[l].expert_ffn(x_dev[l:l + 1], 1)
+
+    with torch.cuda.stream(stream):
+        step()                       # eager pass: sets kernel attributes before capture
+        ffn_only()
+    torch.cuda.synchronize()
+    g_step = _capture(step, stream)
+    g_ffn = _capture(ffn_only, stream)
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            g_step.replay()
+            g_ffn.replay()
+    torch.cuda.synchronize()
+
+    # whole-path timing (clock samples cover a pre-roll, the timed region and a post-roll)
+    sampler = ClockSampler(device.index or 0)
+    sampler.start()
+    with torch.cuda.stream(stream):
+        roll = max(1, int(0.6 / max(_timed_replays(g_step.replay, 3, stream) / 3e3, 1e-6)))
+        _timed_replays(g_step.replay, roll, stream)
+        barrier(world)
+        torch.cuda.synchronize()
+        total_ms = _timed_replays(g_step.replay, steps, stream)
+        barrier(world)
+        _timed_replays(g_step.replay, roll, stream)
+    clocks = sampler.stop()
+    ms_step = total_ms / steps
+
+    # the dominant kernels: the expert FFN of each layer, timed alone (40 per replay)
+    with torch.cuda.stream(stream):
+        ffn_ms = _timed_replays(g_ffn.replay, steps, stream) / (steps * LAYERS)
+    achieved = FFN_BYTES_T1 / (ffn_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "kernel": "moe_expert_ffn (T=1: gate/up + SwiGLU, then down + combine-add)",
+                "algorithmic_bytes": FFN_BYTES_T1, "avg_launch_us": ffn_ms * 1e3,
+                "peak_source": peaks["source"] + " hbm_gbs"}
+
+    # end to end through the public API: pinned host x -> device, 40 layers, y -> pinned host
+    x_pin = torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).pin_memory()
+    y_pin = torch.empty(LAYERS, H, dtype=torch.bfloat16).pin_memory()
+
+    def e2e_step():
+        x_dev.copy_(x_pin, non_blocking=True)
+        g_step.replay()
+        y_pin.copy_(y_dev, non_blocking=True)
+        stream.synchronize()
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            e2e_step()
+        e2e_ms = _timed_replays(e2e_step, steps, stream) / steps
+    e2e = {"value": LAYERS / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": LAYERS * H * 2,
+           "d2h_bytes_per_step": LAYERS * H * 2, "ms_per_step": e2e_ms}
+
+    launches = _launch_count(layers[0], 1) * LAYERS
+    return {"ms_per_step": ms_step, "units_per_step": LAYERS * 1, "roofline": roofline, "e2e": e2e,
+            "clocks": clocks, "gpu_launches": launches * steps, "_host_layers": host}
+
+
+def run_prefill(device, steps, warmup, world, peaks):
+    """T = 2048 prefill layer (uniform router): tokens/s and the expert-FFN tensor roofline."""
+    import torch
+    import gen
+    from bit_dequant_expert_b200.layer import MoELayer, to_device
+    spec = gen.config(3)
+    lay = gen.make_layer(spec)
+    T = spec.T
+    L = MoELayer(lay, max_tokens=T, device=device)
+    x = to_device(lay["x"], device)
+    del lay
+    stream = torch.cuda.Stream(device=device)
+    with torch.cuda.stream(stream):
+        L.forward(x)
+    torch.cuda.synchronize()
+    g = _capture(lambda: L.forward(x), stream)
+    gf = _capture(lambda: L.expert_ffn(x, T), stream)
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            g.replay()
+        ms = _timed_replays(g.replay, steps, stream) / steps
+        for _ in range(warmup):
+            gf.replay()
+        ffn_ms = _timed_replays(gf.replay, steps, stream) / steps
+    rows = (K + 1) * T
+    flops = 2.0 * rows * (2 * I * H + H * I)
+    tflops = flops / (ffn_ms * 1e-3) / 1e12
+    wbytes = (E + 1) * EXPERT_BYTES
+    return {"workload": "prefill: T=2048, uniform router (H 2048, I 512, E 256 top-8 + shared, G 64)",
+            "value": T / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms, "steps": steps,
+            "ffn_ms": ffn_ms,
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": tflops / peaks["bf16_tflops"], "traffic": None,
+                         "kernel": "moe_expert_ffn (T=2048)", "algorithmic_flops": flops,
+                         "peak_source": peaks["source"] + " bf16_tflops (burst)",
+                         "hbm_frac_of_weight_bytes": wbytes / (ffn_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+            "gpu_launches_per_step": _launch_count(L, T),
+            "l2": "inputs larger than L2 (455.8 MB of packed weights per layer)"}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the T=2048 prefill measurement")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle CPU baseline")
+    args = ap.parse_args(argv)
+    warmup = max(args.warmup, 3)
+    world, rank, local = dist_env()
+
+    if args.impl == "reference":
+        return run_reference(args, world, rank, warmup)
+
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", torch.cuda.current_device())
+    peaks = load_peaks()
+
+    res = run_decode(device, args.steps, warmup, world, peaks)
+    pre = None if args.no_prefill else run_prefill(device, max(args.steps // 10, 5), warmup, world, peaks)
+
+    ms, units = aggregate(res["ms_per_step"], res["units_per_step"], world)
+    value = units / (ms / 1e3)
+
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16 (4-bit weights, fp32 accumulation)",
+        "data": "synthetic (seeded; SplitMix64 layers shaped like the pages' model)",
+        "config": {
+            "workload": "decode: T=1 x 40 distinct layers cycled (H 2048, I 512, E 256 top-8 + shared, G 64)",
+            "global_batch": world,
+            "seq_len": 1,
+            "parallelism": "replicas" if world > 1 else "single GPU",
+            "l2": "inputs larger than L2 (18.2 GB of weights streamed per step; no flush)",
+            "graph": "one CUDA graph per step (40 layers x route, permute, ffn, combine)",
+        },
+        "decode_token_per_s": world / (ms / 1e3),
+        "gpu_launches": res["gpu_launches"],
+        "roofline": res["roofline"],
+        "e2e": res["e2e"],
+        "clocks": res["clocks"],
+        "peaks": peaks,
+    }
+    if pre is not None:
+        line["prefill_t2048"] = pre
+    if rank == 0 and world == 1:
+        budget = args.cpu_budget
+        layers_host = res.pop("_host_layers")
+        rate, n, dt = time_oracle_decode(layers_host, budget)
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": omp_threads(), "kind": "oracle",
+                                "sample": "%d layer passes (T=1) of the first decode layers, %.1f s" % (n, dt)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        barrier(world)
+        dist.destroy_process_group()
+    return 0
+
+
+def run_reference(args, world, rank, warmup):
+    """The reference arm: the CPU oracle on this host's cores, same metric."""
+    if rank != 0:
+        return 0
+    import gen
+    spec = gen.config(1)
+    layers = [gen.make_layer(spec, l) for l in range(3)]
+    per_step = []
+    total_t = time.perf_counter()
+    for s in range(warmup + args.steps):
+        t0 = time.perf_counter()
+        # one bounded sample step: one layer pass of T = 1 (of the 40-layer workload)
+        import oracle
+        oracle.layer(layers[s % len(layers)])
+        if s >= warmup:
+            per_step.append(time.perf_counter() - t0)
+        if time.perf_counter() - total_t > 150:
+            break
+    ms = 1e3 * float(np.mean(per_step)) if per_step else float("nan")
+    value = 1e3 / ms
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": len(per_step),
+        "warmup": warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic (seeded)",
+        "config": {"workload": "decode: T=1 x 40 distinct layers cycled (H 2048, I 512, E 256 top-8 + shared, G 64)",
+                   "global_batch": 1, "seq_len": 1, "parallelism": "host cores"},
+        "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": omp_threads(), "kind": "oracle",
+                         "sample": "one layer pass (T=1) per step, layers 0-2 cycled"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,73 @@
+// Host-side launchers of the moe_b200 kernels (internal interface).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+namespace moe {
+
+struct RouterArgs {
+    int T, H, E;
+    const uint16_t* x;
+    const uint16_t* w_router;
+    const float* logits_in;
+    const float* bias;
+    int64_t bias_stride;
+    int32_t* topk_idx;
+    float* topk_w;
+    int32_t* counts;
+    float* logits_ws;   // [T, E] scratch
+    int32_t* err;
+};
+
+struct PermuteArgs {
+    int T, E;
+    const int32_t* topk_idx;
+    const int32_t* counts;
+    int32_t* offsets;
+    int32_t* row_to_pair;
+    int32_t* pair_to_row;
+    uint8_t* scratch;   // permute_ws_bytes(T, E, K)
+    int32_t* err;
+};
+
+struct FfnArgs {
+    int T, H, I, E, K, G, has_shared, mode;
+    const uint16_t* x;
+    const uint32_t* gu_codes;
+    const uint16_t* gu_sb;
+    const uint32_t* d_codes;
+    const uint16_t* d_sb;
+    const int32_t* offsets;
+    const int32_t* row_to_pair;
+    const float* topk_w;
+    uint16_t* h;          // [(K+1) T, I] bf16 scratch: routed rows, then shared rows
+    float* y_acc;         // scatter mode
+    uint16_t* y_rows;     // pairs mode
+    uint16_t* y_shared;   // pairs mode
+    int32_t* err;
+};
+
+struct CombineArgs {
+    int T, H, has_shared, mode;
+    const float* y_acc;
+    const uint16_t* rows;
+    const uint16_t* shared;
+    const int32_t* pair_to_row;
+    const float* w;
+    uint16_t* y;
+    int32_t* err;
+};
+
+cudaError_t launch_router(const RouterArgs& a, cudaStream_t st);
+size_t permute_ws_bytes(int T, int E, int K);
+cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st);
+cudaError_t launch_ffn_simt(const FfnArgs& a, cudaStream_t st);
+cudaError_t launch_ffn_gemv(const FfnArgs& a, cudaStream_t st);
+cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st);
+bool ffn_tc_supported(const FfnArgs& a);
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st);
+
+}  // namespace moe

@@ -1,0 +1,104 @@
+"""Torch-level convenience wrapper: device buffers for one MoE layer and the
+four library calls in order.  Allocation and marshalling only; the compute is
+entirely in libmoe_b200."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import (MOE_MODE_PAIRS, MOE_MODE_SCATTER, MOE_PATH_AUTO, config, moe_combine, moe_expert_ffn_path,
+               moe_permute, moe_route, moe_workspace_init, moe_workspace_size)
+
+
+def to_device(a, device, dtype=None) -> torch.Tensor:
+    """numpy uint16 (bf16 bits) / uint32 / float32 / int32 -> device tensor with the same bytes."""
+    if isinstance(a, torch.Tensor):
+        return a.to(device)
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+    elif a.dtype == np.uint32:
+        t = torch.from_numpy(a.view(np.int32))
+    else:
+        t = torch.from_numpy(a)
+    if dtype is not None:
+        t = t.to(dtype)
+    return t.to(device)
+
+
+class MoELayer:
+    """One layer's weights resident on the device plus its scratch buffers.
+
+    weights: dict with w_router [E,H] bf16 bits, gu_codes [E+1,2I,H/8] u32,
+    gu_sb [E+1,2I,H/G,2] bf16 bits, d_codes [E+1,H,I/8] u32, d_sb
+    [E+1,H,I/G,2] bf16 bits (numpy arrays or device tensors).
+    """
+
+    def __init__(self, weights: dict, max_tokens: int, device="cuda", mode=MOE_MODE_SCATTER,
+                 path=MOE_PATH_AUTO, has_shared=True):
+        gu = weights["gu_codes"]
+        E1, I2, H8 = gu.shape
+        H = H8 * 8
+        I = I2 // 2
+        self.cfg = config(hidden=H, inter=I, num_experts=E1 - 1, top_k=8, group_size=64,
+                          has_shared=1 if has_shared else 0)
+        self.H, self.I, self.E, self.K = H, I, E1 - 1, 8
+        self.device = torch.device(device)
+        self.mode, self.path = mode, path
+        self.max_tokens = max_tokens
+        self.w_router = to_device(weights["w_router"], self.device)
+        self.gu_codes = to_device(weights["gu_codes"], self.device)
+        self.gu_sb = to_device(weights["gu_sb"], self.device)
+        self.d_codes = to_device(weights["d_codes"], self.device)
+        self.d_sb = to_device(weights["d_sb"], self.device)
+        nbytes = moe_workspace_size(self.cfg, max_tokens)
+        if nbytes == 0:
+            raise ValueError("unsupported layer configuration")
+        self.ws = torch.zeros(nbytes, dtype=torch.uint8, device=self.device)
+        moe_workspace_init(self.ws)
+        T, K, E = max_tokens, self.K, self.E
+        dev = self.device
+        self.topk_idx = torch.empty(T, K, dtype=torch.int32, device=dev)
+        self.topk_w = torch.empty(T, K, dtype=torch.float32, device=dev)
+        self.counts = torch.empty(E, dtype=torch.int32, device=dev)
+        self.offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        self.row_to_pair = torch.empty(T * K, dtype=torch.int32, device=dev)
+        self.pair_to_row = torch.empty(T * K, dtype=torch.int32, device=dev)
+        if mode == MOE_MODE_SCATTER:
+            self.out0 = torch.empty(T, H, dtype=torch.float32, device=dev)
+            self.out1 = None
+        else:
+            self.out0 = torch.empty(T * K, H, dtype=torch.bfloat16, device=dev)
+            self.out1 = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+        self.y = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+
+    def route(self, x, T, logit_bias=None, bias_stride=0, logits_in=None, stream=None):
+        moe_route(self.cfg, T, x, self.w_router, logits_in, logit_bias, bias_stride, self.topk_idx, self.topk_w,
+                  self.counts, self.ws, stream=stream)
+
+    def permute(self, T, stream=None):
+        moe_permute(self.cfg, T, self.topk_idx, self.counts, self.offsets, self.row_to_pair, self.pair_to_row,
+                    self.ws, stream=stream)
+
+    def expert_ffn(self, x, T, stream=None, path=None):
+        moe_expert_ffn_path(self.cfg, T, x, self.gu_codes, self.gu_sb, self.d_codes, self.d_sb, self.offsets,
+                            self.row_to_pair, self.topk_w, self.mode, self.out0, self.out1, self.ws,
+                            self.path if path is None else path, stream=stream)
+
+    def combine(self, T, stream=None, y_out=None):
+        y = self.y if y_out is None else y_out
+        moe_combine(self.cfg, T, self.mode, self.out0, self.out1, self.pair_to_row, self.topk_w, y,
+                    stream=stream)
+
+    def forward(self, x: torch.Tensor, logit_bias=None, bias_stride=0, logits_in=None, stream=None,
+                y_out=None) -> torch.Tensor:
+        """y [T, H] bf16 for x [T, H] bf16 (written to y_out if given, else to
+        the layer's own output buffer, a view of which is returned)."""
+        T = x.shape[0]
+        if T > self.max_tokens:
+            raise ValueError("T=%d exceeds max_tokens=%d" % (T, self.max_tokens))
+        self.route(x, T, logit_bias, bias_stride, logits_in, stream)
+        self.permute(T, stream)
+        self.expert_ffn(x, T, stream)
+        self.combine(T, stream, y_out)
+        return self.y[:T] if y_out is None else y_out

@@ -1,0 +1,194 @@
+/*
+ * moe_b200: one mixture-of-experts layer with groupwise-affine 4-bit expert
+ * weights, for NVIDIA B200 (sm_100a).  C ABI.
+ *
+ * The layer (the Lily pages: "Perplexity's Lily brings fast local AI to Apple
+ * silicon Macs", sections "A 35B Model Built for Local Memory" and "Where the
+ * Engine Gains Speed"; "Perplexity built an inference engine for one model,
+ * one chip", second and third paragraphs):
+ *   a router scores E = 256 experts per token, keeps the top k = 8 and
+ *   renormalises their softmax weights; one shared expert sees every token;
+ *   every expert is a SwiGLU FFN whose weights are 4-bit codes with a bf16
+ *   (scale, bias) per group of G = 64 inputs, reconstructed inside the
+ *   expert GEMM tile by tile; the outputs are combined with the routing
+ *   weights.  Routing never returns to the host.
+ *
+ * The layer is four calls on one CUDA stream:
+ *   moe_route -> moe_permute -> moe_expert_ffn -> moe_combine.
+ *
+ * Conventions for every call:
+ *  - All pointers are DEVICE pointers unless stated otherwise; the caller
+ *    owns every buffer.  The library allocates nothing, frees nothing and
+ *    keeps no global state.  Tensors are row-major and contiguous.  bf16
+ *    values travel as uint16_t bit patterns.
+ *  - Alignment: every pointer 16-byte aligned; the packed weight arrays
+ *    (codes and scale/bias) and the workspace 256-byte aligned.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *    are asynchronous and never synchronise the host, except
+ *    moe_get_device_error.
+ *  - Host-side problems (null pointer, unsupported shape, small workspace)
+ *    return an error before anything is launched.  Device-side problems
+ *    (non-finite logit, routing index out of range, an expired bounded
+ *    wait) set a sticky error word in the workspace and the kernels carry
+ *    on with safe values; moe_get_device_error reads it.
+ *  - Concurrent calls must use distinct workspaces.
+ *
+ * Supported shapes: hidden % 256 == 0, inter % 128 == 0, num_experts == 256,
+ * top_k == 8, group_size == 64, has_shared in {0, 1}, 1 <= T <= 65536.
+ * Anything else returns MOE_ERR_UNSUPPORTED.
+ *
+ * Packed weights of an [N, K] matrix (N outputs, K inputs), matrices of all
+ * experts stacked, shared expert last (index num_experts):
+ *   codes [n_mat][N][K/8] uint32: nibble j (bits 4j..4j+3) of word m holds the
+ *         unsigned code q of input 8m + j;
+ *   sb    [n_mat][N][K/G][2] bf16: (scale, bias) of the group of G inputs;
+ *   weight(n, k) = scale * q + bias.
+ * gate_up matrices are [2I, H] (gate rows 0..I-1, up rows I..2I-1); down
+ * matrices are [H, I].
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1, /* null pointer, T < 1, bad mode */
+    MOE_ERR_UNSUPPORTED = 2, /* shape outside the supported set */
+    MOE_ERR_WORKSPACE = 3,   /* workspace too small or misaligned */
+    MOE_ERR_CUDA = 4,        /* a CUDA runtime call failed */
+    MOE_ERR_NONFINITE = 5,   /* device: NaN or Inf among a token's logits */
+    MOE_ERR_TIMEOUT = 6,     /* device: a bounded wait expired */
+    MOE_ERR_BOUNDS = 7       /* device: routing index out of range or repeated */
+} moe_status_t;
+
+typedef struct {
+    int32_t hidden;      /* H */
+    int32_t inter;       /* I, expert intermediate size */
+    int32_t num_experts; /* E routed experts */
+    int32_t top_k;       /* k */
+    int32_t group_size;  /* G inputs per (scale, bias) pair */
+    int32_t has_shared;  /* 1: matrix index E is the always-on shared expert */
+} moe_config_t;
+
+/* Output modes of moe_expert_ffn / moe_combine. */
+#define MOE_MODE_SCATTER 0 /* out0 = y_acc fp32 [T, H]: weighted sum accumulated in place */
+#define MOE_MODE_PAIRS 1   /* out0 = y_rows bf16 [T*k, H] per routed row, out1 = y_shared bf16 [T, H] */
+
+/* Expert-FFN implementations for moe_expert_ffn_path (0 chooses by shape). */
+#define MOE_PATH_AUTO 0
+#define MOE_PATH_SIMT 1    /* CUDA-core dequant + dot products, any T */
+#define MOE_PATH_GEMV 2    /* memory-bound split-K GEMV, few rows per expert */
+#define MOE_PATH_TC 3      /* TMA + in-smem dequant + tcgen05 MMA into TMEM */
+
+/* Bytes of workspace that the calls need for up to max_tokens tokens; 0 if
+ * the configuration is unsupported.  Caller allocates it (256-byte aligned)
+ * and zero-fills it once, or calls moe_workspace_init. */
+size_t moe_workspace_size(const moe_config_t* cfg, int32_t max_tokens);
+
+/* Clears the workspace's sticky error word (async on stream). */
+int32_t moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Router (the pages: "a router picks eight subnetworks out of 256"; "GPU-
+ * resident expert routing").
+ *   x          bf16 [T, H] activations.
+ *   w_router   bf16 [E, H] router weights.
+ *   logits_in  nullable fp32 [T, E]: when given, used instead of x . w_router^T
+ *              (x and w_router may then be NULL).
+ *   logit_bias nullable fp32, row t at logit_bias + t * logit_bias_row_stride
+ *              (stride 0: one [E] row for every token); added once.
+ * Logits are fp32 in a fixed order (the contract order): slice s in 0..31
+ * owns the 8-input chunks c = s, s+32, ...; acc[s] = fma(x, w, acc[s]) over
+ * its chunks in order, inputs ascending within a chunk; then an xor
+ * butterfly over the slices (offsets 16, 8, 4, 2, 1); then + bias.
+ * Outputs:
+ *   topk_idx  int32 [T, k]: the k largest logits, ordered by (logit desc,
+ *             expert asc); -0.0 == +0.0.
+ *   topk_w    fp32  [T, k]: softmax of the selected logits (== the 256-way
+ *             softmax restricted to them and renormalised).
+ *   counts    int32 [E]: tokens routed to each expert.
+ * A token with a non-finite logit sets MOE_ERR_NONFINITE and is routed to
+ * experts 0..k-1 with weight 1/k.
+ */
+int32_t moe_route(const moe_config_t* cfg, int32_t T, const uint16_t* x, const uint16_t* w_router,
+                  const float* logits_in, const float* logit_bias, int64_t logit_bias_row_stride,
+                  int32_t* topk_idx, float* topk_w, int32_t* counts, void* ws, size_t ws_bytes,
+                  void* stream);
+
+/*
+ * Token permutation: stable expert-major order of the T*k (token, slot)
+ * pairs, pair p = t*k + slot.
+ *   counts      nullable int32 [E] from moe_route; when given it is checked
+ *               against topk_idx (mismatch sets MOE_ERR_BOUNDS).
+ *   offsets     int32 [E+1]: exclusive scan of the counts, offsets[E] = T*k.
+ *   row_to_pair int32 [T*k]: rows offsets[e]..offsets[e+1]-1 hold expert e's
+ *               pairs in increasing token order.
+ *   pair_to_row int32 [T*k]: inverse of row_to_pair.
+ * An index outside 0..E-1 or an expert repeated within a token sets
+ * MOE_ERR_BOUNDS.
+ */
+int32_t moe_permute(const moe_config_t* cfg, int32_t T, const int32_t* topk_idx, const int32_t* counts,
+                    int32_t* offsets, int32_t* row_to_pair, int32_t* pair_to_row, void* ws,
+                    size_t ws_bytes, void* stream);
+
+/*
+ * Expert FFNs (the pages: "reconstructs weights inside the grouped GEMM, one
+ * tile at a time"; "one shared expert sees everything"): for every row r of
+ * expert e with token t,
+ *   h = silu(x_t . Wg_e^T) * (x_t . Wu_e^T)  (h rounded to bf16),
+ *   y_r = h . Wd_e^T,
+ * plus the shared expert on every token when cfg->has_shared.  Weights are
+ * dequantised to bf16 on chip; accumulation is fp32.
+ *   gu_codes/gu_sb  packed gate_up matrices, E (+1 shared) of [2I, H].
+ *   d_codes/d_sb    packed down matrices, E (+1 shared) of [H, I].
+ *   offsets, row_to_pair from moe_permute; topk_w from moe_route.
+ *   mode MOE_MODE_SCATTER: out0 = y_acc fp32 [T, H] is overwritten with
+ *        sum_slot w * y_row (+ y_shared); out1 unused.
+ *   mode MOE_MODE_PAIRS: out0 = bf16 [T*k, H] row outputs (row order),
+ *        out1 = bf16 [T, H] shared-expert outputs (unused without shared).
+ */
+int32_t moe_expert_ffn(const moe_config_t* cfg, int32_t T, const uint16_t* x, const uint32_t* gu_codes,
+                       const uint16_t* gu_sb, const uint32_t* d_codes, const uint16_t* d_sb,
+                       const int32_t* offsets, const int32_t* row_to_pair, const float* topk_w,
+                       int32_t mode, void* out0, void* out1, void* ws, size_t ws_bytes, void* stream);
+
+/* moe_expert_ffn with an explicit implementation (MOE_PATH_*). */
+int32_t moe_expert_ffn_path(const moe_config_t* cfg, int32_t T, const uint16_t* x,
+                            const uint32_t* gu_codes, const uint16_t* gu_sb, const uint32_t* d_codes,
+                            const uint16_t* d_sb, const int32_t* offsets, const int32_t* row_to_pair,
+                            const float* topk_w, int32_t mode, void* out0, void* out1, void* ws,
+                            size_t ws_bytes, int32_t path, void* stream);
+
+/*
+ * Combine into the layer output y bf16 [T, H].
+ *   MOE_MODE_SCATTER: in0 = y_acc fp32 [T, H]; y = bf16(y_acc).
+ *   MOE_MODE_PAIRS:   in0 = row outputs bf16 [T*k, H], in1 = shared outputs
+ *                     bf16 [T, H] (ignored without shared);
+ *                     y[t] = bf16(sum_slot w[t,slot] * in0[pair_to_row[t*k+slot]]
+ *                                 + in1[t]), summed in fp32 in slot order.
+ */
+int32_t moe_combine(const moe_config_t* cfg, int32_t T, int32_t mode, const void* in0, const void* in1,
+                    const int32_t* pair_to_row, const float* topk_w, uint16_t* y, void* stream);
+
+/* Synchronises `stream` and returns the workspace's sticky device error
+ * (MOE_OK if none), or MOE_ERR_CUDA if the synchronisation failed. */
+int32_t moe_get_device_error(const void* ws, void* stream);
+
+/* Number of kernels the four calls launch for one layer of T tokens with the
+ * router computing the logits (memsets excluded); -1 if unsupported. */
+int32_t moe_launch_count(const moe_config_t* cfg, int32_t T, int32_t mode, int32_t path);
+
+/* Human-readable name of a status code (static string). */
+const char* moe_status_string(int32_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

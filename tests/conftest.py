@@ -14,3 +14,13 @@ if HERE not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long-running CPU test")
+
+
+def pytest_sessionstart(session):
+    """Build the CUDA library, the generator and the oracle if they are stale."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("_moe_cuda_build",
+                                                  os.path.join(ROOT, "bit_dequant_expert_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build(force=False)

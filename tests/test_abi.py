@@ -1,0 +1,82 @@
+"""The C ABI library on the host: it loads, exports every declared entry
+point, and rejects bad arguments before launching anything (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_b200.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(moe_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_layer_calls():
+    names = declared_functions()
+    for n in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_workspace_size",
+              "moe_get_device_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    import bit_dequant_expert_b200 as m
+    lib = ctypes.CDLL(m.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(declared_functions()) <= set(m.EXPORTED) | {"moe_status_string"}
+
+
+def test_workspace_size_and_config_checks():
+    import bit_dequant_expert_b200 as m
+    cfg = m.config()
+    n1, n2 = m.moe_workspace_size(cfg, 1), m.moe_workspace_size(cfg, 2048)
+    assert 0 < n1 < n2 and n1 % 256 == 0 and n2 % 256 == 0
+    # (k+1) T I bf16 rows of h, T E fp32 logits at least
+    assert n2 >= 9 * 2048 * 512 * 2 + 2048 * 256 * 4
+    for bad in (m.config(hidden=300), m.config(inter=100), m.config(num_experts=128), m.config(top_k=4),
+                m.config(group_size=32), m.config(has_shared=2)):
+        assert m.moe_workspace_size(bad, 16) == 0
+    assert m.moe_workspace_size(cfg, 0) == 0
+    assert m.moe_workspace_size(cfg, 65537) == 0
+
+
+FAKE = 0x7F0000000000   # 256-byte aligned, never dereferenced: every case fails validation first
+
+
+def _route(cfg, T, ws_bytes, ws=FAKE, idx=FAKE, x=FAKE):
+    import bit_dequant_expert_b200 as m
+    return m.moe_route(cfg, T, x, FAKE, None, None, 0, idx, FAKE, FAKE, ws, ws_bytes=ws_bytes, stream=0,
+                       raise_on_error=False)
+
+
+def test_host_validation_before_launch():
+    import bit_dequant_expert_b200 as m
+    cfg = m.config()
+    need = m.moe_workspace_size(cfg, 64)
+    assert _route(cfg, 0, need) == m.MOE_ERR_INVALID_ARG
+    assert _route(m.config(hidden=1000), 64, need) == m.MOE_ERR_UNSUPPORTED
+    assert _route(cfg, 64, need - 256) == m.MOE_ERR_WORKSPACE
+    assert _route(cfg, 64, need, ws=FAKE + 16) == m.MOE_ERR_WORKSPACE
+    assert _route(cfg, 64, need, ws=None) == m.MOE_ERR_WORKSPACE
+    assert _route(cfg, 64, need, idx=None) == m.MOE_ERR_INVALID_ARG
+    assert _route(cfg, 64, need, x=FAKE + 2) == m.MOE_ERR_INVALID_ARG
+    st = m.moe_permute(cfg, 64, FAKE, None, None, FAKE, FAKE, FAKE, ws_bytes=need, stream=0, raise_on_error=False)
+    assert st == m.MOE_ERR_INVALID_ARG
+    st = m.moe_expert_ffn(cfg, 64, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 7, FAKE, FAKE, FAKE,
+                          ws_bytes=need, stream=0, raise_on_error=False)
+    assert st == m.MOE_ERR_INVALID_ARG
+    st = m.moe_expert_ffn(cfg, 64, FAKE, FAKE + 16, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, FAKE, None, FAKE,
+                          ws_bytes=need, stream=0, raise_on_error=False)
+    assert st == m.MOE_ERR_INVALID_ARG      # packed weights must be 256-byte aligned
+    st = m.moe_expert_ffn_path(cfg, 64, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, FAKE, None, FAKE, 0,
+                               ws_bytes=need, stream=0, raise_on_error=False)
+    assert st == m.MOE_ERR_INVALID_ARG      # pairs mode with a shared expert needs out1
+    st = m.moe_combine(cfg, 64, 1, FAKE, FAKE, None, FAKE, FAKE, stream=0, raise_on_error=False)
+    assert st == m.MOE_ERR_INVALID_ARG
+    assert m.moe_get_device_error(None, 0) == m.MOE_ERR_WORKSPACE
+    assert m.moe_status_string(m.MOE_ERR_NONFINITE) == "MOE_ERR_NONFINITE"

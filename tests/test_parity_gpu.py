@@ -1,0 +1,183 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on
+seeded synthetic layers.  Routing, counts and permutations bit-exact; weights
+within 2e-6; outputs within 1e-2 row-relative error."""
+import numpy as np
+import pytest
+
+import gen
+import oracle
+from gpu_util import (check_output, check_permutation_props, check_routing, run_layer, row_rel_err)
+
+pytestmark = pytest.mark.gpu
+
+SCATTER, PAIRS = 0, 1
+SIMT, GEMV, TC = 1, 2, 3
+
+_layers = {}
+
+
+def layer_of(cfg_id, T=None, layer=0):
+    key = (cfg_id, layer)
+    if key not in _layers:
+        spec = gen.config(cfg_id)
+        _layers[key] = gen.make_layer(spec, layer)
+    lay = _layers[key]
+    if T is not None and T != lay["x"].shape[0]:
+        spec = gen.config(cfg_id).with_T(T)
+        lay = dict(lay, **gen.make_activations(spec, layer))
+    return lay
+
+
+def _sample_tokens(T, n, seed):
+    rng = np.random.default_rng(seed)
+    if T <= n:
+        return np.arange(T)
+    return np.sort(np.concatenate([[0, T - 1], rng.choice(np.arange(1, T - 1), n - 2, replace=False)]))
+
+
+@pytest.mark.parametrize("mode", [SCATTER, PAIRS])
+def test_config0_full(mode):
+    lay = layer_of(0)
+    out, _ = run_layer(lay, mode, SIMT)
+    assert out["err"] == 0
+    idx_ref = check_routing(out, lay)
+    counts, offsets, r2p, p2r = oracle.permute(idx_ref, 256)
+    assert np.array_equal(out["counts"], counts) and np.array_equal(out["offsets"], offsets)
+    assert np.array_equal(out["r2p"], r2p) and np.array_equal(out["p2r"], p2r)
+    check_output(out, lay, np.arange(8))
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 5, 7, 8, 33, 257, 4097])
+def test_edge_T_small_shapes(T):
+    lay = layer_of(0, T=T)
+    out, _ = run_layer(lay, SCATTER, SIMT)
+    assert out["err"] == 0
+    idx_ref = check_routing(out, lay)
+    counts, offsets, r2p, p2r = oracle.permute(idx_ref, 256)
+    assert np.array_equal(out["offsets"], offsets) and np.array_equal(out["r2p"], r2p)
+    assert np.array_equal(out["p2r"], p2r)
+    check_output(out, lay, _sample_tokens(T, 24, T))
+
+
+@pytest.mark.parametrize("cfg_id", [2, 3])
+@pytest.mark.parametrize("mode", [SCATTER, PAIRS])
+def test_prefill_configs_simt(cfg_id, mode):
+    lay = layer_of(cfg_id)
+    T = lay["x"].shape[0]
+    out, _ = run_layer(lay, mode, SIMT)
+    assert out["err"] == 0
+    idx_ref = check_routing(out, lay)
+    counts, offsets, r2p, p2r = oracle.permute(idx_ref, 256)
+    assert np.array_equal(out["offsets"], offsets) and np.array_equal(out["r2p"], r2p)
+    check_output(out, lay, _sample_tokens(T, 12, cfg_id))
+
+
+def test_config4_hot_routing_and_sampled_output():
+    lay = layer_of(4)
+    T = lay["x"].shape[0]
+    out, _ = run_layer(lay, SCATTER, SIMT)
+    assert out["err"] == 0
+    tok = _sample_tokens(T, 48, 4)
+    check_routing(out, lay, tokens=tok)
+    check_permutation_props(out, T)
+    hot = set(gen.hot_experts(gen.config(4)).tolist())
+    biased = np.nonzero(lay["logit_bias"].any(axis=1))[0]
+    assert all(set(out["idx"][t].tolist()) == hot for t in biased[:256])
+    check_output(out, lay, tok[:8])
+
+
+def test_config1_decode_layers():
+    spec = gen.config(1)
+    for layer in (0, 17, 39):
+        lay = gen.make_layer(spec, layer)
+        out, _ = run_layer(lay, SCATTER, SIMT)
+        assert out["err"] == 0
+        check_routing(out, lay)
+        check_output(out, lay, [0])
+
+
+def test_logits_in_ties_bitexact():
+    lay = layer_of(0, T=64)
+    rng = np.random.default_rng(1)
+    li = rng.integers(0, 3, size=(64, 256)).astype(np.float32)      # mass ties
+    li[5] = 0.0
+    li[6, ::2] = -0.0                                                 # +0 / -0 ties
+    li[7] = rng.standard_normal(256).astype(np.float32)
+    out, _ = run_layer(lay, SCATTER, SIMT, logits_in=li)
+    assert out["err"] == 0
+    idx_ref, w_ref = oracle.select(li, 8)
+    assert np.array_equal(out["idx"], idx_ref)
+    assert np.abs(out["w"] - w_ref).max() <= 2e-6
+    assert out["idx"][5].tolist() == list(range(8))
+    check_output(out, lay, np.arange(0, 64, 7), logits_in=li)
+
+
+def test_all_tokens_one_expert_set():
+    lay = dict(layer_of(0, T=300))
+    hot = np.array([9, 3, 77, 200, 150, 31, 64, 128])
+    bias = np.zeros(256, dtype=np.float32)
+    bias[hot] = 100.0
+    lay["logit_bias"], lay["bias_stride"] = bias, 0
+    out, _ = run_layer(lay, SCATTER, SIMT)
+    assert out["err"] == 0
+    assert np.all(np.sort(out["idx"], axis=1) == np.sort(hot))
+    assert out["counts"][hot].tolist() == [300] * 8 and out["counts"].sum() == 2400
+    check_permutation_props(out, 300)
+    check_output(out, lay, [0, 1, 150, 299])
+
+
+def test_nonfinite_logit_sets_error():
+    import bit_dequant_expert_b200 as m
+    lay = layer_of(0, T=16)
+    li = np.zeros((16, 256), dtype=np.float32)
+    li[3, 100] = np.nan
+    li[9, 7] = np.inf
+    out, L = run_layer(lay, SCATTER, SIMT, logits_in=li)
+    assert out["err"] == m.MOE_ERR_NONFINITE
+    assert out["idx"][3].tolist() == list(range(8)) and np.all(out["w"][3] == 0.125)
+    # the error is sticky until the workspace is re-initialised
+    assert m.moe_get_device_error(L.ws) == m.MOE_ERR_NONFINITE
+    m.moe_workspace_init(L.ws)
+    assert m.moe_get_device_error(L.ws) == 0
+
+
+def test_permute_rejects_bad_routing():
+    import torch
+    import bit_dequant_expert_b200 as m
+    cfg = m.config(hidden=512, inter=128)
+    T = 4
+    ws = torch.zeros(m.moe_workspace_size(cfg, T), dtype=torch.uint8, device="cuda")
+    idx = torch.tensor([[0, 1, 2, 3, 4, 5, 6, 7]] * T, dtype=torch.int32, device="cuda")
+    idx[2, 5] = 3          # repeated expert in a token
+    off = torch.empty(257, dtype=torch.int32, device="cuda")
+    r2p = torch.empty(T * 8, dtype=torch.int32, device="cuda")
+    p2r = torch.empty(T * 8, dtype=torch.int32, device="cuda")
+    m.moe_permute(cfg, T, idx, None, off, r2p, p2r, ws)
+    assert m.moe_get_device_error(ws) == m.MOE_ERR_BOUNDS
+    m.moe_workspace_init(ws)
+    idx[2, 5] = 300        # out of range
+    m.moe_permute(cfg, T, idx, None, off, r2p, p2r, ws)
+    assert m.moe_get_device_error(ws) == m.MOE_ERR_BOUNDS
+
+
+@pytest.mark.parametrize("T", [1, 100, 256, 257, 1000, 5000])
+def test_permute_bitexact_random(T):
+    import torch
+    import bit_dequant_expert_b200 as m
+    cfg = m.config(hidden=512, inter=128)
+    rng = np.random.default_rng(T)
+    idx = np.stack([rng.permutation(256)[:8] for _ in range(T)]).astype(np.int32)
+    if T >= 1000:
+        idx[: T // 2] = np.arange(8)          # skew: half the tokens on experts 0..7
+    counts, offsets, r2p, p2r = oracle.permute(idx, 256)
+    ws = torch.zeros(m.moe_workspace_size(cfg, T), dtype=torch.uint8, device="cuda")
+    d_idx = torch.from_numpy(idx).cuda()
+    d_cnt = torch.from_numpy(counts).cuda()
+    off = torch.empty(257, dtype=torch.int32, device="cuda")
+    g_r2p = torch.empty(T * 8, dtype=torch.int32, device="cuda")
+    g_p2r = torch.empty(T * 8, dtype=torch.int32, device="cuda")
+    m.moe_permute(cfg, T, d_idx, d_cnt, off, g_r2p, g_p2r, ws)
+    assert m.moe_get_device_error(ws) == 0
+    assert np.array_equal(off.cpu().numpy(), offsets)
+    assert np.array_equal(g_r2p.cpu().numpy(), r2p)
+    assert np.array_equal(g_p2r.cpu().numpy(), p2r)
