@@ -43,7 +43,10 @@ MOE_PATH_TC = 3
 EXPORTED = (
     "moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permute", "moe_expert_ffn",
     "moe_expert_ffn_path", "moe_combine", "moe_get_device_error", "moe_status_string", "moe_launch_count",
+    "moe_permute_static",
 )
+
+MOE_STATIC_MAX_TOKENS = 16384
 
 
 class moe_config_t(ctypes.Structure):
@@ -76,6 +79,8 @@ _lib.moe_combine.restype = _I32
 _lib.moe_combine.argtypes = [_CFG, _I32, _I32, _P, _P, _P, _P, _P, _P]
 _lib.moe_get_device_error.restype = _I32
 _lib.moe_get_device_error.argtypes = [_P, _P]
+_lib.moe_permute_static.restype = _I32
+_lib.moe_permute_static.argtypes = [_CFG, _I32, _P, _P, _P, _P, _P, _P, _P]
 _lib.moe_launch_count.restype = _I32
 _lib.moe_launch_count.argtypes = [_CFG, _I32, _I32, _I32]
 _lib.moe_status_string.restype = ctypes.c_char_p
@@ -167,6 +172,15 @@ def moe_combine(cfg, T, mode, in0, in1, pair_to_row, topk_w, y, stream=None, rai
     st = _lib.moe_combine(ctypes.byref(cfg), T, mode, _ptr(in0), _ptr(in1), _ptr(pair_to_row), _ptr(topk_w), _ptr(y),
                           _stream(stream))
     return _check(st, "moe_combine", raise_on_error)
+
+
+def moe_permute_static(cfg, T, topk_idx, counts, offsets, row_to_pair, pair_to_row, err_out=None, stream=None,
+                       raise_on_error=True) -> int:
+    """moe_permute without a workspace, for callers that cannot allocate
+    device memory (scratch lives in a fixed array inside the library)."""
+    st = _lib.moe_permute_static(ctypes.byref(cfg), T, _ptr(topk_idx), _ptr(counts), _ptr(offsets),
+                                 _ptr(row_to_pair), _ptr(pair_to_row), _ptr(err_out), _stream(stream))
+    return _check(st, "moe_permute_static", raise_on_error)
 
 
 def moe_launch_count(cfg, T, mode=MOE_MODE_SCATTER, path=MOE_PATH_AUTO) -> int:

@@ -180,6 +180,34 @@ int32_t moe_combine(const moe_config_t* cfg, int32_t T, int32_t mode, const void
  * (MOE_OK if none), or MOE_ERR_CUDA if the synchronisation failed. */
 int32_t moe_get_device_error(const void* ws, void* stream);
 
+/*
+ * moe_permute_static: moe_permute for callers that cannot allocate device
+ * memory.  The Lily pages have no counterpart to this call; it exists for
+ * callers with no way to obtain scratch memory: a plugin inside a host
+ * runtime that owns every device allocation and hands it only pre-allocated
+ * input and output buffers, a real-time path where cudaMalloc (which can
+ * synchronise the device) is not allowed, or a deployment whose device
+ * memory is budgeted by another allocator.
+ *
+ * Same inputs, outputs and results as moe_permute, without a workspace: the
+ * scratch (chunk histograms and ranks) lives in a fixed device array inside
+ * the library, MOE_STATIC_MAX_TOKENS tokens' worth (576 KiB), which every GPU
+ * that loads the library holds until the process exits.  The call allocates
+ * and frees nothing.
+ *   err_out  nullable device int32: zeroed by the call, then receives the
+ *            call's device error (MOE_ERR_BOUNDS) if any.
+ * T > MOE_STATIC_MAX_TOKENS returns MOE_ERR_UNSUPPORTED before any launch.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  All calls share the one array, which keeps the previous call's
+ * contents: calls that overlap on the GPU (other streams, other host threads
+ * on the same device) race on it and must be serialised by the caller.
+ */
+#define MOE_STATIC_MAX_TOKENS 16384
+int32_t moe_permute_static(const moe_config_t* cfg, int32_t T, const int32_t* topk_idx, const int32_t* counts,
+                           int32_t* offsets, int32_t* row_to_pair, int32_t* pair_to_row, int32_t* err_out,
+                           void* stream);
+
 /* Number of kernels the four calls launch for one layer of T tokens with the
  * router computing the logits (memsets excluded); -1 if unsupported. */
 int32_t moe_launch_count(const moe_config_t* cfg, int32_t T, int32_t mode, int32_t path);
