@@ -284,9 +284,30 @@ def run_decode(device, steps, warmup, world, peaks):
     e2e = {"value": LAYERS / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": LAYERS * H * 2,
            "d2h_bytes_per_step": LAYERS * H * 2, "ms_per_step": e2e_ms}
 
+    breakdown = _breakdown(layers, [x_dev[l:l + 1] for l in range(LAYERS)], 1, steps, stream)
     launches = _launch_count(layers[0], 1) * LAYERS
     return {"ms_per_step": ms_step, "units_per_step": LAYERS * 1, "roofline": roofline, "e2e": e2e,
-            "clocks": clocks, "gpu_launches": launches * steps, "_host_layers": host}
+            "clocks": clocks, "gpu_launches": launches * steps, "breakdown_us_per_layer": breakdown,
+            "_host_layers": host}
+
+
+def _breakdown(layers, xs, T, steps, stream):
+    """Device time per layer of each of the four calls, each captured alone (us)."""
+    import torch
+    parts = {
+        "route": lambda: [L.route(x, T) for L, x in zip(layers, xs)],
+        "permute": lambda: [L.permute(T) for L in layers],
+        "expert_ffn": lambda: [L.expert_ffn(x, T) for L, x in zip(layers, xs)],
+        "combine": lambda: [L.combine(T) for L in layers],
+    }
+    out = {}
+    for name, fn in parts.items():
+        g = _capture(fn, stream)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                g.replay()
+            out[name] = 1e3 * _timed_replays(g.replay, steps, stream) / (steps * len(layers))
+    return out
 
 
 def run_prefill(device, steps, warmup, world, peaks):
@@ -313,6 +334,7 @@ def run_prefill(device, steps, warmup, world, peaks):
         for _ in range(warmup):
             gf.replay()
         ffn_ms = _timed_replays(gf.replay, steps, stream) / steps
+    breakdown = _breakdown([L], [x], T, steps, stream)
     rows = (K + 1) * T
     flops = 2.0 * rows * (2 * I * H + H * I)
     tflops = flops / (ffn_ms * 1e-3) / 1e12
@@ -326,6 +348,7 @@ def run_prefill(device, steps, warmup, world, peaks):
                          "peak_source": peaks["source"] + " bf16_tflops (burst)",
                          "hbm_frac_of_weight_bytes": wbytes / (ffn_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
             "gpu_launches_per_step": _launch_count(L, T),
+            "breakdown_us": breakdown,
             "l2": "inputs larger than L2 (455.8 MB of packed weights per layer)"}
 
 
@@ -381,6 +404,7 @@ def main(argv=None):
             "graph": "one CUDA graph per step (40 layers x route, permute, ffn, combine)",
         },
         "decode_token_per_s": world / (ms / 1e3),
+        "breakdown_us_per_layer": res["breakdown_us_per_layer"],
         "gpu_launches": res["gpu_launches"],
         "roofline": res["roofline"],
         "e2e": res["e2e"],

@@ -12,11 +12,14 @@ constexpr int kWarp = 32;
 
 // ------------------------------------------------------------------ layout
 
-// Workspace header: sticky error word at byte 0; the rest of the first 256
-// bytes are reserved.  Scratch sections follow, 256-byte aligned.
+// Workspace header: sticky error word at byte 0, the decode kernel's grid
+// barrier counter at byte 8 (monotonic, 64-bit); the rest of the first 256
+// bytes is reserved.  Scratch sections follow, 256-byte aligned.
 struct WsHeader {
     int32_t error;
-    int32_t reserved[63];
+    int32_t pad;
+    unsigned long long grid_sync;
+    int32_t reserved[60];
 };
 
 __host__ __device__ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -64,17 +67,24 @@ __device__ __forceinline__ uint32_t ldg_u32(const void* p) {
     return v;
 }
 
-// Raises a kernel's dynamic shared-memory limit once per device (kernel
-// attributes are per device; setting them is kept out of stream capture).
+// Raises a kernel's dynamic shared-memory limit when a launch needs more than
+// was set before on this device (kernel attributes are per device; after the
+// first launch of each size the call is skipped, so it stays out of stream
+// capture).  `set_bytes` is a per-kernel table of 64 devices.
 template <typename Kern>
-inline cudaError_t set_smem_once(Kern* k, int bytes, unsigned long long* done_mask) {
+inline cudaError_t set_smem_once(Kern* k, int bytes, int* set_bytes) {
     int dev = 0;
     cudaError_t ce = cudaGetDevice(&dev);
     if (ce != cudaSuccess) return ce;
-    const unsigned long long bit = 1ull << (dev & 63);
-    if (__atomic_load_n(done_mask, __ATOMIC_ACQUIRE) & bit) return cudaSuccess;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (__atomic_load_n(&set_bytes[dev], __ATOMIC_ACQUIRE) >= bytes) return cudaSuccess;
     ce = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (ce == cudaSuccess) __atomic_fetch_or(done_mask, bit, __ATOMIC_ACQ_REL);
+    if (ce == cudaSuccess) {
+        int cur = __atomic_load_n(&set_bytes[dev], __ATOMIC_ACQUIRE);
+        while (cur < bytes && !__atomic_compare_exchange_n(&set_bytes[dev], &cur, bytes, false, __ATOMIC_ACQ_REL,
+                                                           __ATOMIC_ACQUIRE)) {
+        }
+    }
     return ce;
 }
 

@@ -267,9 +267,9 @@ cudaError_t launch_ffn_simt(const FfnArgs& a, cudaStream_t st) {
     {
         dim3 grid(ntiles, (a.I + 31) / 32);
         const size_t sm = pre + (size_t)R * a.H * sizeof(uint16_t);
-        static unsigned long long done = 0;
+        static int done[64] = {0};
         if (sm > 48 * 1024) {
-            cudaError_t ce = set_smem_once(k_ffn1_simt<R>, (int)sm, &done);
+            cudaError_t ce = set_smem_once(k_ffn1_simt<R>, (int)sm, done);
             if (ce != cudaSuccess) return ce;
         }
         k_ffn1_simt<R><<<grid, 256, sm, st>>>(a);
@@ -277,9 +277,9 @@ cudaError_t launch_ffn_simt(const FfnArgs& a, cudaStream_t st) {
     {
         dim3 grid(ntiles, (a.H + 31) / 32);
         const size_t sm = pre + (size_t)R * a.I * sizeof(uint16_t);
-        static unsigned long long done = 0;
+        static int done[64] = {0};
         if (sm > 48 * 1024) {
-            cudaError_t ce = set_smem_once(k_ffn2_simt<R>, (int)sm, &done);
+            cudaError_t ce = set_smem_once(k_ffn2_simt<R>, (int)sm, done);
             if (ce != cudaSuccess) return ce;
         }
         k_ffn2_simt<R><<<grid, 256, sm, st>>>(a);

@@ -65,7 +65,8 @@ cudaError_t launch_router(const RouterArgs& a, cudaStream_t st);
 size_t permute_ws_bytes(int T, int E, int K);
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st);
 cudaError_t launch_ffn_simt(const FfnArgs& a, cudaStream_t st);
-cudaError_t launch_ffn_gemv(const FfnArgs& a, cudaStream_t st);
+bool ffn_gemv_supported(const FfnArgs& a);
+cudaError_t launch_ffn_gemv(const FfnArgs& a, unsigned long long* sync, cudaStream_t st);
 cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st);
 bool ffn_tc_supported(const FfnArgs& a);
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st);

@@ -52,6 +52,25 @@ int32_t* err_word(void* ws) { return reinterpret_cast<int32_t*>(ws); }
 
 int32_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
+// Implementation chosen for MOE_PATH_AUTO: the memory-bound decode kernel for
+// a handful of tokens, otherwise the general CUDA-core path.
+int32_t resolve_path(const FfnArgs& a) {
+    if (ffn_gemv_supported(a)) return MOE_PATH_GEMV;
+    return MOE_PATH_SIMT;
+}
+
+FfnArgs shape_only(const moe_config_t* cfg, int32_t T) {
+    FfnArgs a = {};
+    a.T = T;
+    a.H = cfg->hidden;
+    a.I = cfg->inter;
+    a.E = cfg->num_experts;
+    a.K = cfg->top_k;
+    a.G = cfg->group_size;
+    a.has_shared = cfg->has_shared;
+    return a;
+}
+
 }  // namespace
 
 extern "C" {
@@ -157,14 +176,17 @@ int32_t moe_expert_ffn_path(const moe_config_t* cfg, int32_t T, const uint16_t* 
     a.y_shared = mode == MOE_MODE_PAIRS ? static_cast<uint16_t*>(out1) : nullptr;
     a.err = err_word(ws);
     cudaStream_t s = (cudaStream_t)stream;
-    if (mode == MOE_MODE_SCATTER) {
-        cudaError_t ce = cudaMemsetAsync(a.y_acc, 0, sizeof(float) * (size_t)T * a.H, s);
-        if (ce != cudaSuccess) return MOE_ERR_CUDA;
-    }
+    if (path == MOE_PATH_AUTO) path = resolve_path(a);
     switch (path) {
-        case MOE_PATH_AUTO:
         case MOE_PATH_SIMT:
+            if (mode == MOE_MODE_SCATTER) {
+                cudaError_t ce = cudaMemsetAsync(a.y_acc, 0, sizeof(float) * (size_t)T * a.H, s);
+                if (ce != cudaSuccess) return MOE_ERR_CUDA;
+            }
             return cuda_status(launch_ffn_simt(a, s));
+        case MOE_PATH_GEMV:
+            if (!ffn_gemv_supported(a)) return MOE_ERR_UNSUPPORTED;
+            return cuda_status(launch_ffn_gemv(a, &reinterpret_cast<WsHeader*>(ws)->grid_sync, s));
         default:
             return MOE_ERR_UNSUPPORTED;
     }
@@ -218,10 +240,12 @@ int32_t moe_launch_count(const moe_config_t* cfg, int32_t T, int32_t mode, int32
     if (mode != MOE_MODE_SCATTER && mode != MOE_MODE_PAIRS) return -1;
     const int route = 2;
     const int permute = T <= 256 ? 1 : 3;
+    const FfnArgs a = shape_only(cfg, T);
+    if (path == MOE_PATH_AUTO) path = resolve_path(a);
     int ffn;
     switch (path) {
-        case MOE_PATH_AUTO:
         case MOE_PATH_SIMT: ffn = 2; break;
+        case MOE_PATH_GEMV: if (!ffn_gemv_supported(a)) return -1; ffn = 1; break;
         default: return -1;
     }
     return route + permute + ffn + 1;
