@@ -1,0 +1,587 @@
+// Expert FFNs for prefill: grouped GEMMs on the 5th-generation tensor cores
+// with the 4-bit dequantisation fused into the main loop.
+//
+// Lily pages: "Perplexity's Lily brings fast local AI to Apple silicon Macs",
+// section "Where the Engine Gains Speed" (weights reconstructed inside the
+// grouped GEMM, one tile at a time; expert GEMMs take about 90% of prefill);
+// "Perplexity built an inference engine for one model, one chip", third
+// paragraph (folding the dequantisation into the matrix multiplication so an
+// expanded array never touches memory: +77.4% prefill at 512 tokens).
+//
+// One persistent kernel template, instantiated for gate/up (+SwiGLU) and for
+// down (+weighted combine).  A tile is 128 weight rows (MMA M) x up to 128
+// token rows (MMA N) of one expert; K runs in 64-input chunks, one (scale,
+// bias) group each.  Per chunk:
+//   warp 0       TMA: the tile's 128 rows x 64 codes (4 KB) and the B operand
+//                rows (x rows already gathered into expert order for gate/up,
+//                h rows for down; contiguous either way) into one smem ring
+//                stage; B lands 128B-swizzled and K-major, as the MMA reads it;
+//   warps 2-3    down: each tile's per-column token and routing weight, built
+//                one tile ahead of the epilogue;
+//   warps 4-11   dequantise codes to bf16 (scale * q + bias) and write them as
+//                the A operand straight into tensor memory (tcgen05.st), so
+//                the MMA reads only B from shared memory;
+//   warp 1       one thread issues 4 tcgen05.mma (K = 16 each) into one of two
+//                TMEM accumulators and commits to mbarriers;
+//   warps 12-15  epilogue from TMEM: SwiGLU (gate and up rows interleaved on
+//                adjacent TMEM lanes) -> h in bf16, or w * y scattered into
+//                y_acc (fp32 red) / bf16 rows.
+// Every wait is bounded (error word MOE_ERR_TIMEOUT, never a hang).
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kThreads = 512;
+constexpr int kNT = 128;                 // token rows per tile (MMA N, max)
+constexpr int kBK = 64;                  // inputs per chunk = one (scale, bias) group
+constexpr int kStages = 8;
+constexpr int kCodesStage = 128 * 32;    // 128 rows x 64 nibbles
+constexpr int kBStage = kNT * 128;       // kNT rows x 64 bf16
+constexpr int kACol0 = 2 * kNT;          // TMEM: two fp32 accumulators, then the A stages
+constexpr int kAStageCols = kBK / 2;     // bf16 pairs per 32-bit column
+constexpr int kTmemCols = 512;
+constexpr int kTabs = 4;                 // column tables in flight (down epilogue)
+constexpr int kSbBytes = 16384;          // one tile's (scale, bias) words: 128 rows x up to 32 groups
+static_assert(kACol0 + kStages * kAStageCols <= kTmemCols, "TMEM budget");
+
+struct Smem {
+    uint8_t b[kStages][kBStage];                 // offset 0, 1024-aligned
+    uint8_t codes[kStages][kCodesStage];
+    uint32_t sbs[2][kSbBytes / 4];               // per-tile (scale, bias) rows, double-buffered
+    uint64_t full[kStages], a_full[kStages], mma_done[kStages];
+    uint64_t acc_full[2], acc_empty[2], tab_full[kTabs], tab_empty[kTabs], sb_full[2], sb_empty[2];
+    int tok[kTabs][kNT];
+    float w[kTabs][kNT];
+    int pre[260];
+    int off[260];                                // offsets[0..E], cached
+    uint32_t tmem_base;
+};
+
+struct TcArgs {
+    FfnArgs f;
+    int gateup;      // 1: gate/up + SwiGLU; 0: down + combine
+};
+
+struct Tile {
+    int e, r0, nr, npad, mb;   // expert (E = shared), first row, rows, rows padded to 16, M block
+    size_t hrow0;              // first h row of the tile
+};
+
+__device__ __forceinline__ int tiles_per_block_row(const FfnArgs& a, int gateup) {
+    return gateup ? a.I / 64 : a.H / 128;
+}
+
+// Prefix of tiles per expert: pre[e] first tile of expert e, pre[E] first
+// shared tile, pre[E+1] total.  blockDim.x >= E.
+__device__ void tile_prefix(const FfnArgs& a, int gateup, int* pre, int* off) {
+    __shared__ int warp_tot[32];
+    const int MB = tiles_per_block_row(a, gateup);
+    const int e = threadIdx.x;
+    int tiles = 0;
+    if (e < a.E) {
+        int lo = a.offsets[e], hi = a.offsets[e + 1];
+        if (lo < 0 || hi < lo || hi > a.T * a.K) {
+            set_error(a.err, MOE_ERR_BOUNDS);
+            lo = hi = 0;
+        }
+        tiles = (hi - lo + kNT - 1) / kNT * MB;
+        off[e] = lo;
+        if (e == a.E - 1) off[a.E] = hi;
+    }
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int inc = tiles;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xFFFFFFFFu, inc, off);
+        if (lane >= off) inc += o;
+    }
+    if (lane == 31) warp_tot[warp] = inc;
+    __syncthreads();
+    int base = 0;
+    for (int w = 0; w < warp; ++w) base += warp_tot[w];
+    if (e < a.E) pre[e] = base + inc - tiles;
+    if (threadIdx.x == blockDim.x - 1) {
+        const int routed = base + inc;
+        pre[a.E] = routed;
+        pre[a.E + 1] = routed + (a.has_shared ? (a.T + kNT - 1) / kNT * MB : 0);
+    }
+    __syncthreads();
+}
+
+__device__ __forceinline__ Tile decode_tile(const FfnArgs& a, int gateup, const int* pre, const int* off, int t) {
+    const int MB = tiles_per_block_row(a, gateup);
+    Tile tl;
+    int e;
+    if (t >= pre[a.E]) {
+        e = a.E;
+    } else {
+        int lo = 0, hi = a.E - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (pre[mid] <= t) lo = mid; else hi = mid - 1;
+        }
+        e = lo;
+    }
+    const int local = t - pre[e];
+    const int tb = local / MB;
+    tl.e = e;
+    tl.mb = local % MB;
+    if (e == a.E) {
+        tl.r0 = tb * kNT;
+        tl.nr = min(kNT, a.T - tl.r0);
+        tl.hrow0 = (size_t)a.T * a.K + tl.r0;
+    } else {
+        tl.r0 = off[e] + tb * kNT;
+        tl.nr = min(kNT, (e + 1 < a.E ? off[e + 1] : off[a.E]) - tl.r0);
+        tl.hrow0 = tl.r0;
+    }
+    tl.npad = (tl.nr + 15) & ~15;
+    return tl;
+}
+
+// First weight row (within the packed matrices) of the tile's two 64-row
+// halves (gate/up) or of its 128 rows (down).
+__device__ __forceinline__ int wrow_gate(const FfnArgs& a, const Tile& tl) { return tl.e * 2 * a.I + 64 * tl.mb; }
+__device__ __forceinline__ int wrow_up(const FfnArgs& a, const Tile& tl) { return tl.e * 2 * a.I + a.I + 64 * tl.mb; }
+__device__ __forceinline__ int wrow_down(const FfnArgs& a, const Tile& tl) { return tl.e * a.H + 128 * tl.mb; }
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_ffn_tc(const __grid_constant__ CUtensorMap codes_map, const __grid_constant__ CUtensorMap b_map,
+             const __grid_constant__ CUtensorMap sb_map, const TcArgs ta) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // the 128B-swizzled B stages need a 1024-byte aligned base
+    Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const FfnArgs& a = ta.f;
+    const int gateup = ta.gateup;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int K = gateup ? a.H : a.I;            // reduction length of this GEMM
+    const int KC = K / kBK;                      // chunks per tile
+    const int ngroups = K / 64;
+    // (scale, bias) rows go through shared memory by TMA when a row's words
+    // span whole 16-byte units; otherwise (tiny K) each thread reads its own
+    const bool sb_tma = (ngroups & 3) == 0;
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.a_full[s], 8);
+            mbar_init(&sm.mma_done[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.acc_full[b], 1);
+            mbar_init(&sm.acc_empty[b], 4);
+        }
+        for (int b = 0; b < kTabs; ++b) {
+            mbar_init(&sm.tab_full[b], 2);
+            mbar_init(&sm.tab_empty[b], 4);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.sb_full[b], 1);
+            mbar_init(&sm.sb_empty[b], 8);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm.tmem_base, kTmemCols);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    // y_acc is accumulated by the down launch; the gate/up launch (which runs
+    // before it on the stream) zeroes it.
+    if (gateup && a.mode == MOE_MODE_SCATTER) {
+        const size_t n4 = (size_t)a.T * a.H / 4, per = (n4 + gridDim.x - 1) / gridDim.x;
+        const size_t lo = blockIdx.x * per, hi = min(n4, lo + per);
+        for (size_t q = lo + tid; q < hi; q += kThreads)
+            reinterpret_cast<float4*>(a.y_acc)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    tile_prefix(a, gateup, sm.pre, sm.off);   // contains __syncthreads
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    const int ntiles = sm.pre[a.E + 1];
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        // Stage s is refilled once the MMAs of its previous use completed (which
+        // implies its codes were dequantised).  B: one or two 64-row boxes.
+        // The whole next tile's codes and (scale, bias) rows are pulled into L2
+        // while this one streams, so the ring's TMA loads hit L2: a ring of a
+        // few 4 KB stages alone keeps too few bytes in flight for HBM.
+        auto prefetch_tile = [&](int t) {
+            if (t >= ntiles || lane != 0) return;
+            const Tile tl = decode_tile(a, gateup, sm.pre, sm.off, t);
+            const uint8_t* codes = reinterpret_cast<const uint8_t*>(gateup ? a.gu_codes : a.d_codes);
+            const uint8_t* sbb = reinterpret_cast<const uint8_t*>(gateup ? a.gu_sb : a.d_sb);
+            if (gateup) {
+                prefetch_l2(codes + (size_t)wrow_gate(a, tl) * (a.H / 2), 64 * (a.H / 2));
+                prefetch_l2(codes + (size_t)wrow_up(a, tl) * (a.H / 2), 64 * (a.H / 2));
+                prefetch_l2(sbb + (size_t)wrow_gate(a, tl) * (a.H / 16), 64 * (a.H / 16));
+                prefetch_l2(sbb + (size_t)wrow_up(a, tl) * (a.H / 16), 64 * (a.H / 16));
+            } else {
+                prefetch_l2(codes + (size_t)wrow_down(a, tl) * (a.I / 2), 128 * (a.I / 2));
+                prefetch_l2(sbb + (size_t)wrow_down(a, tl) * (a.I / 16), 128 * (a.I / 16));
+            }
+        };
+        prefetch_tile(blockIdx.x);
+        uint32_t it = 0, lt = 0;
+        for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
+            const Tile tl = decode_tile(a, gateup, sm.pre, sm.off, t);
+            prefetch_tile(t + gridDim.x);
+            if (sb_tma && lane == 0) {
+                const int buf = lt & 1;
+                if (lt >= 2) mbar_wait_bounded(&sm.sb_empty[buf], ((lt >> 1) - 1) & 1, a.err);
+                mbar_arrive_expect_tx(&sm.sb_full[buf], 128 * ngroups * 4);
+                if (gateup) {
+                    tma_load_2d(sm.sbs[buf], &sb_map, 0, wrow_gate(a, tl), &sm.sb_full[buf]);
+                    tma_load_2d(sm.sbs[buf] + 64 * ngroups, &sb_map, 0, wrow_up(a, tl), &sm.sb_full[buf]);
+                } else {
+                    tma_load_2d(sm.sbs[buf], &sb_map, 0, wrow_down(a, tl), &sm.sb_full[buf]);
+                }
+            }
+            const int nbox = tl.npad > 64 ? 2 : 1;
+            for (int kc = 0; kc < KC; ++kc, ++it) {
+                const int s = it % kStages;
+                if (lane == 0) {
+                    if (it >= kStages) mbar_wait_bounded(&sm.mma_done[s], ((it / kStages) - 1) & 1, a.err);
+                    mbar_arrive_expect_tx(&sm.full[s], kCodesStage + nbox * 64 * 128);
+                    if (gateup) {
+                        tma_load_2d(sm.codes[s], &codes_map, kc * 8, wrow_gate(a, tl), &sm.full[s]);
+                        tma_load_2d(sm.codes[s] + kCodesStage / 2, &codes_map, kc * 8, wrow_up(a, tl), &sm.full[s]);
+                    } else {
+                        tma_load_2d(sm.codes[s], &codes_map, kc * 8, wrow_down(a, tl), &sm.full[s]);
+                    }
+                    for (int bx = 0; bx < nbox; ++bx)
+                        tma_load_2d(sm.b[s] + bx * 64 * 128, &b_map, kc * kBK, (int)tl.hrow0 + 64 * bx, &sm.full[s]);
+                }
+                __syncwarp();
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            uint32_t it = 0, lt = 0;
+            for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
+                const Tile tl = decode_tile(a, gateup, sm.pre, sm.off, t);
+                const int ab = lt & 1;
+                if (lt >= 2) mbar_wait_bounded(&sm.acc_empty[ab], ((lt >> 1) - 1) & 1, a.err);
+                tc_fence_after();
+                const uint32_t idesc = idesc_bf16_f32(128, tl.npad);
+                const uint32_t d_tmem = tmem + ab * kNT;
+                for (int kc = 0; kc < KC; ++kc, ++it) {
+                    const int s = it % kStages;
+                    const uint32_t par = (it / kStages) & 1;
+                    mbar_wait_bounded(&sm.a_full[s], par, a.err);
+                    mbar_wait_bounded(&sm.full[s], par, a.err);
+                    tc_fence_after();
+                    const uint64_t bdesc = smem_desc_sw128(smem_u32(sm.b[s]));
+                    const uint32_t a_tmem = tmem + kACol0 + s * kAStageCols;
+#pragma unroll
+                    for (int j = 0; j < kBK / 16; ++j)
+                        tc_mma_ts(d_tmem, a_tmem + 8 * j, bdesc + 2 * j, idesc, (kc | j) != 0);
+                    tc_commit(&sm.mma_done[s]);
+                }
+                tc_commit(&sm.acc_full[ab]);
+            }
+        }
+    } else if (warp < 4) {
+        // ------------------------------------------------------------ column tables (down)
+        if (!gateup) {
+            const int bt = tid - 64;
+            uint32_t lt = 0;
+            for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
+                const Tile tl = decode_tile(a, gateup, sm.pre, sm.off, t);
+                const int slot = lt % kTabs;
+                if (lt >= kTabs) mbar_wait_bounded(&sm.tab_empty[slot], ((lt / kTabs) - 1) & 1, a.err);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int c = bt + 64 * h;
+                    int tok = 0;
+                    float w = 0.0f;
+                    if (c < tl.nr) {
+                        if (tl.e == a.E) {
+                            tok = tl.r0 + c;
+                            w = 1.0f;
+                        } else {
+                            const int p = a.row_to_pair[tl.r0 + c];
+                            if (p >= 0 && p < a.T * a.K) {
+                                tok = p / a.K;
+                                w = a.topk_w[p];
+                            } else {
+                                set_error(a.err, MOE_ERR_BOUNDS);
+                            }
+                        }
+                    }
+                    sm.tok[slot][c] = tok;
+                    sm.w[slot][c] = w;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.tab_full[slot]);
+            }
+        }
+    } else if (warp < 12) {
+        // ------------------------------------------------------------ dequantisers
+        const int q = warp & 3;              // TMEM lane quadrant
+        const int khalf = (warp - 4) >> 2;   // which 32 inputs of the chunk
+        const int L = 32 * q + lane;         // A row == TMEM lane
+        const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16) + kACol0 + 16 * khalf;
+        const uint32_t* sbase = reinterpret_cast<const uint32_t*>(gateup ? a.gu_sb : a.d_sb);
+        // codes of row L inside a stage: gate/up interleave gate and up rows on
+        // adjacent lanes (even: gate, odd: up), so SwiGLU pairs are lane pairs
+        const int srow_off = gateup ? ((L & 1) * (kCodesStage / 2) + (L >> 1) * 32) : L * 32;
+        uint32_t it = 0, lt = 0;
+        for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
+            const Tile tl = decode_tile(a, gateup, sm.pre, sm.off, t);
+            const int wrow = gateup ? ((L & 1) ? wrow_up(a, tl) : wrow_gate(a, tl)) + (L >> 1) : wrow_down(a, tl) + L;
+            const uint32_t* sbrow = sbase + (size_t)wrow * ngroups;
+            const int buf = lt & 1;
+            // this row's (scale, bias) words in shared memory: gate rows 0..63, up rows 64..127
+            const uint32_t* sbs_row = sm.sbs[buf] + (size_t)(gateup ? ((L & 1) * 64 + (L >> 1)) : L) * ngroups;
+            if (sb_tma) mbar_wait_bounded(&sm.sb_full[buf], (lt >> 1) & 1, a.err);
+            uint4 cur = make_uint4(0, 0, 0, 0);
+            auto sb_of = [&](int kc) -> uint32_t {
+                if (!sb_tma) return ldg_u32(sbrow + kc);
+                const int r = kc & 3;
+                if (r == 0) cur = *reinterpret_cast<const uint4*>(sbs_row + kc);
+                return r == 0 ? cur.x : r == 1 ? cur.y : r == 2 ? cur.z : cur.w;
+            };
+            auto dequant16 = [&](uint4 cw, uint32_t sbw, uint32_t (&v)[16]) {
+                const uint32_t s2 = prmt(sbw, sbw, 0x1010), b2 = prmt(sbw, sbw, 0x3232);
+                const uint32_t wds[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const uint32_t w0 = wds[m], w4 = w0 >> 4;
+                    v[4 * m + 0] = dequant_pair<0>(w0, w4, s2, b2);
+                    v[4 * m + 1] = dequant_pair<1>(w0, w4, s2, b2);
+                    v[4 * m + 2] = dequant_pair<2>(w0, w4, s2, b2);
+                    v[4 * m + 3] = dequant_pair<3>(w0, w4, s2, b2);
+                }
+            };
+            // two chunks per round: one tensor-memory store wait covers both
+            for (int kc = 0; kc < KC; kc += 2, it += 2) {
+                const int s0 = it % kStages, s1 = (it + 1) % kStages;
+                const uint32_t sb0 = sb_of(kc), sb1 = sb_of(kc + 1);
+                mbar_wait_bounded(&sm.full[s0], (it / kStages) & 1, a.err);
+                const uint4 cw0 = *reinterpret_cast<const uint4*>(sm.codes[s0] + srow_off + 16 * khalf);
+                mbar_wait_bounded(&sm.full[s1], ((it + 1) / kStages) & 1, a.err);
+                const uint4 cw1 = *reinterpret_cast<const uint4*>(sm.codes[s1] + srow_off + 16 * khalf);
+                uint32_t v0[16], v1[16];
+                dequant16(cw0, sb0, v0);
+                dequant16(cw1, sb1, v1);
+                if (it >= kStages) mbar_wait_bounded(&sm.mma_done[s0], ((it / kStages) - 1) & 1, a.err);
+                if (it + 1 >= kStages) mbar_wait_bounded(&sm.mma_done[s1], (((it + 1) / kStages) - 1) & 1, a.err);
+                tc_fence_after();
+                tmem_st16(lane_addr + s0 * kAStageCols, v0);
+                tmem_st16(lane_addr + s1 * kAStageCols, v1);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&sm.a_full[s0]);
+                    mbar_arrive(&sm.a_full[s1]);
+                }
+            }
+            if (sb_tma) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.sb_empty[buf]);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;
+        uint32_t lt = 0;
+        for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
+            const Tile tl = decode_tile(a, gateup, sm.pre, sm.off, t);
+            const int ab = lt & 1;
+            const int slot = lt % kTabs;
+            if (!gateup) mbar_wait_bounded(&sm.tab_full[slot], (lt / kTabs) & 1, a.err);
+            mbar_wait_bounded(&sm.acc_full[ab], (lt >> 1) & 1, a.err);
+            tc_fence_after();
+            const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + ab * kNT;
+            for (int c0 = 0; c0 < tl.npad; c0 += 16) {
+                uint32_t v[16];
+                tmem_ld16(taddr + c0, v);
+                tmem_ld_wait();
+                if (gateup) {
+                    // lanes 2i / 2i+1 hold gate / up of row j = 64 mb + 16 q + i; the
+                    // even lane finishes the even columns, the odd lane the odd ones
+                    const int j = 64 * tl.mb + 16 * q + (lane >> 1);
+                    const int odd = lane & 1;
+#pragma unroll
+                    for (int c = 0; c < 16; c += 2) {
+                        const float m0 = __uint_as_float(v[c]), m1 = __uint_as_float(v[c + 1]);
+                        // even lane sends column c+1, odd lane sends column c
+                        const float recv = __shfl_xor_sync(0xFFFFFFFFu, odd ? m0 : m1, 1);
+                        const float gate = odd ? recv : m0;       // column c + odd
+                        const float up = odd ? m1 : recv;
+                        const int col = c0 + c + odd;
+                        if (col < tl.nr) {
+                            const float hval = __fdividef(gate, 1.0f + __expf(-gate)) * up;
+                            a.h[(tl.hrow0 + col) * a.I + j] = f32_to_bf16(hval);
+                        }
+                    }
+                } else {
+                    const int n = 128 * tl.mb + 32 * q + lane;
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const int col = c0 + c;
+                        if (col >= tl.nr) break;
+                        const float y = __uint_as_float(v[c]);
+                        if (a.mode == MOE_MODE_SCATTER) {
+                            atomicAdd(a.y_acc + (size_t)sm.tok[slot][col] * a.H + n, sm.w[slot][col] * y);
+                        } else if (tl.e == a.E) {
+                            a.y_shared[(size_t)(tl.r0 + col) * a.H + n] = f32_to_bf16(y);
+                        } else {
+                            a.y_rows[(size_t)(tl.r0 + col) * a.H + n] = f32_to_bf16(y);
+                        }
+                    }
+                }
+            }
+            if (!gateup) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.tab_empty[slot]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.acc_empty[ab]);
+        }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------ host side
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_fn() {
+    static EncodeTiled fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiled>(p);
+    }
+    return fn;
+}
+
+// Packed codes of n_mat stacked [N, K] matrices as a 2-D tensor of u32 words
+// (K/8 per row), read in boxes of 8 words x box_rows rows.
+bool make_codes_map(CUtensorMap* m, const uint32_t* codes, int rows, int K, int box_rows) {
+    EncodeTiled enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)(K / 8), (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+    const cuuint32_t box[2] = {8, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(codes), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 [rows, cols] activations read in boxes of 64 columns (128 bytes) x
+// box_rows rows, 128B-swizzled (the K-major layout the MMA reads).
+bool make_act_map(CUtensorMap* m, const uint16_t* base, int rows, int cols, int box_rows) {
+    EncodeTiled enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// (scale, bias) words of stacked [N, K] matrices: rows of K/64 u32, read
+// in boxes of all K/64 words x box_rows rows.
+bool make_sb_map(CUtensorMap* m, const uint16_t* sb, int rows, int K, int box_rows) {
+    EncodeTiled enc = encode_fn();
+    if (!enc) return false;
+    const int ng = K / 64;
+    const cuuint64_t dims[2] = {(cuuint64_t)ng, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)ng * 4};
+    const cuuint32_t box[2] = {(cuuint32_t)ng, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint16_t*>(sb), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+    static int sms[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (!sms[dev]) cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+    return sms[dev];
+}
+
+// xg[r] = x[token of row r]: routed rows in expert order (row_to_pair), then
+// the shared expert's rows (tokens 0..T-1).  One warp per row, 16-byte moves.
+__global__ void __launch_bounds__(256) k_gather_rows(FfnArgs a) {
+    const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    const int rows = (a.K + 1) * a.T;
+    if (row >= rows) return;
+    int tok;
+    if (row >= a.T * a.K) {
+        tok = row - a.T * a.K;
+    } else {
+        const int p = a.row_to_pair[row];
+        tok = (p >= 0 && p < a.T * a.K) ? p / a.K : 0;
+        if (p < 0 || p >= a.T * a.K) set_error(a.err, MOE_ERR_BOUNDS);
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)tok * a.H);
+    uint4* dst = reinterpret_cast<uint4*>(a.xg + (size_t)row * a.H);
+    for (int c = lane; c < a.H / 8; c += 32) dst[c] = src[c];
+}
+
+}  // namespace
+
+bool ffn_tc_supported(const FfnArgs& a) {
+    // chunks are taken two at a time: K/64 even for both GEMMs
+    // one tile's (scale, bias) rows must fit their shared-memory buffer
+    return a.E <= 256 && a.K == 8 && a.G == 64 && a.H % 128 == 0 && a.I % 128 == 0 && a.H >= 128 && a.I >= 128 &&
+           128 * (a.H / 64) * 4 <= kSbBytes && 128 * (a.I / 64) * 4 <= kSbBytes;
+}
+
+cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
+    const int nmat = a.E + 1;
+    CUtensorMap gu_map, d_map, x_map, h_map;
+    if (!make_codes_map(&gu_map, a.gu_codes, nmat * 2 * a.I, a.H, 64)) return cudaErrorInvalidValue;
+    if (!make_codes_map(&d_map, a.d_codes, nmat * a.H, a.I, 128)) return cudaErrorInvalidValue;
+    if (!make_act_map(&x_map, a.xg, (a.K + 1) * a.T, a.H, 64)) return cudaErrorInvalidValue;
+    if (!make_act_map(&h_map, a.h, (a.K + 1) * a.T, a.I, 64)) return cudaErrorInvalidValue;
+    // (scale, bias) maps only when a row's words fill whole 16-byte units
+    CUtensorMap gsb_map = gu_map, dsb_map = d_map;
+    if ((a.H / 64) % 4 == 0 && !make_sb_map(&gsb_map, a.gu_sb, nmat * 2 * a.I, a.H, 64)) return cudaErrorInvalidValue;
+    if ((a.I / 64) % 4 == 0 && !make_sb_map(&dsb_map, a.d_sb, nmat * a.H, a.I, 128)) return cudaErrorInvalidValue;
+    const int grows = (a.K + 1) * a.T;
+    k_gather_rows<<<(grows + 7) / 8, 256, 0, st>>>(a);
+    const int smem = (int)sizeof(Smem) + 1024;
+    static int done[64] = {0};
+    cudaError_t ce = set_smem_once(k_ffn_tc, smem, done);
+    if (ce != cudaSuccess) return ce;
+    const int G = num_sms();
+    if (G <= 0) return cudaErrorInvalidDevice;
+    TcArgs ta;
+    ta.f = a;
+    ta.gateup = 1;
+    k_ffn_tc<<<G, kThreads, smem, st>>>(gu_map, x_map, gsb_map, ta);
+    ce = cudaGetLastError();
+    if (ce != cudaSuccess) return ce;
+    ta.gateup = 0;
+    k_ffn_tc<<<G, kThreads, smem, st>>>(d_map, h_map, dsb_map, ta);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

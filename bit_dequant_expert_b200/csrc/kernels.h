@@ -44,6 +44,7 @@ struct FfnArgs {
     const int32_t* row_to_pair;
     const float* topk_w;
     uint16_t* h;          // [(K+1) T, I] bf16 scratch: routed rows, then shared rows
+    uint16_t* xg;         // [(K+1) T, H] bf16 scratch: x rows in the same row order (tensor-core path)
     float* y_acc;         // scatter mode
     uint16_t* y_rows;     // pairs mode
     uint16_t* y_shared;   // pairs mode

@@ -18,7 +18,7 @@ bool config_ok(const moe_config_t* c) {
 }
 
 struct WsLayout {
-    size_t logits, perm, h, total;
+    size_t logits, perm, h, xg, total;
 };
 
 WsLayout layout(const moe_config_t* c, int T) {
@@ -30,6 +30,8 @@ WsLayout layout(const moe_config_t* c, int T) {
     off += permute_ws_bytes(T, c->num_experts, c->top_k);
     L.h = off;
     off += align256((size_t)(c->top_k + 1) * T * c->inter * sizeof(uint16_t));
+    L.xg = off;
+    off += align256((size_t)(c->top_k + 1) * T * c->hidden * sizeof(uint16_t));
     L.total = off;
     return L;
 }
@@ -56,6 +58,7 @@ int32_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_
 // a handful of tokens, otherwise the general CUDA-core path.
 int32_t resolve_path(const FfnArgs& a) {
     if (ffn_gemv_supported(a)) return MOE_PATH_GEMV;
+    if (ffn_tc_supported(a)) return MOE_PATH_TC;
     return MOE_PATH_SIMT;
 }
 
@@ -171,6 +174,7 @@ int32_t moe_expert_ffn_path(const moe_config_t* cfg, int32_t T, const uint16_t* 
     a.row_to_pair = row_to_pair;
     a.topk_w = topk_w;
     a.h = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + layout(cfg, T).h);
+    a.xg = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + layout(cfg, T).xg);
     a.y_acc = mode == MOE_MODE_SCATTER ? static_cast<float*>(out0) : nullptr;
     a.y_rows = mode == MOE_MODE_PAIRS ? static_cast<uint16_t*>(out0) : nullptr;
     a.y_shared = mode == MOE_MODE_PAIRS ? static_cast<uint16_t*>(out1) : nullptr;
@@ -187,6 +191,9 @@ int32_t moe_expert_ffn_path(const moe_config_t* cfg, int32_t T, const uint16_t* 
         case MOE_PATH_GEMV:
             if (!ffn_gemv_supported(a)) return MOE_ERR_UNSUPPORTED;
             return cuda_status(launch_ffn_gemv(a, &reinterpret_cast<WsHeader*>(ws)->grid_sync, s));
+        case MOE_PATH_TC:
+            if (!ffn_tc_supported(a)) return MOE_ERR_UNSUPPORTED;
+            return cuda_status(launch_ffn_tc(a, s));
         default:
             return MOE_ERR_UNSUPPORTED;
     }
@@ -246,6 +253,7 @@ int32_t moe_launch_count(const moe_config_t* cfg, int32_t T, int32_t mode, int32
     switch (path) {
         case MOE_PATH_SIMT: ffn = 2; break;
         case MOE_PATH_GEMV: if (!ffn_gemv_supported(a)) return -1; ffn = 1; break;
+        case MOE_PATH_TC: if (!ffn_tc_supported(a)) return -1; ffn = 3; break;
         default: return -1;
     }
     return route + permute + ffn + 1;

@@ -237,3 +237,62 @@ def test_gemv_all_tokens_same_experts():
     out, _ = run_layer(lay, SCATTER, GEMV)
     assert out["err"] == 0
     check_output(out, lay, np.arange(8))
+
+
+# ------------------------------------------------------------ tensor-core (tcgen05) path
+
+
+@pytest.mark.parametrize("mode", [SCATTER, PAIRS])
+@pytest.mark.parametrize("T", [8, 33, 300])
+def test_tc_small_shapes(T, mode):
+    lay = layer_of(0, T=T)
+    out, _ = run_layer(lay, mode, TC)
+    assert out["err"] == 0
+    check_routing(out, lay)
+    check_output(out, lay, _sample_tokens(T, 24, T))
+
+
+@pytest.mark.parametrize("cfg_id", [2, 3])
+@pytest.mark.parametrize("mode", [SCATTER, PAIRS])
+def test_tc_prefill_configs(cfg_id, mode):
+    lay = layer_of(cfg_id)
+    T = lay["x"].shape[0]
+    out, _ = run_layer(lay, mode, TC)
+    assert out["err"] == 0
+    check_routing(out, lay)
+    check_output(out, lay, _sample_tokens(T, 16, cfg_id + 10))
+
+
+def test_tc_config4_hot():
+    lay = layer_of(4)
+    T = lay["x"].shape[0]
+    out, _ = run_layer(lay, SCATTER, TC)
+    assert out["err"] == 0
+    tok = _sample_tokens(T, 24, 44)
+    check_routing(out, lay, tokens=tok)
+    check_permutation_props(out, T)
+    check_output(out, lay, tok[:10])
+
+
+@pytest.mark.parametrize("T", [1, 17, 4097])
+def test_tc_and_simt_against_oracle(T):
+    """The same layer through the tensor-core and CUDA-core paths (pairs mode,
+    deterministic): each within the layer tolerance of the oracle on sampled
+    tokens, the tensor-core path repeatable bit for bit, and the two within
+    2e-2 of each other everywhere (two approximations each within 1e-2 of the
+    oracle can differ by up to twice that)."""
+    from bit_dequant_expert_b200.layer import MoELayer, to_device
+    lay = layer_of(3, T=T)
+    Lt = MoELayer(lay, max_tokens=T, path=TC, mode=PAIRS)
+    Ls = MoELayer(lay, max_tokens=T, path=SIMT, mode=PAIRS)
+    x = to_device(lay["x"], "cuda")
+    yt = Lt.forward(x).float().cpu().numpy().astype(np.float64)
+    ys = Ls.forward(x).float().cpu().numpy().astype(np.float64)
+    again = Lt.forward(x).float().cpu().numpy().astype(np.float64)
+    import bit_dequant_expert_b200 as m
+    assert m.moe_get_device_error(Lt.ws) == 0
+    assert np.array_equal(yt, again)
+    assert np.max(row_rel_err(yt, ys)) < 2e-2
+    tok = _sample_tokens(T, 12, T + 5)
+    check_output(dict(y=yt), lay, tok)
+    check_output(dict(y=ys), lay, tok)
