@@ -314,11 +314,13 @@ def run_prefill(device, steps, warmup, world, peaks):
     """T = 2048 prefill layer (uniform router): tokens/s and the expert-FFN tensor roofline."""
     import torch
     import gen
+    from bit_dequant_expert_b200 import MOE_MODE_PAIRS
     from bit_dequant_expert_b200.layer import MoELayer, to_device
     spec = gen.config(3)
     lay = gen.make_layer(spec)
     T = spec.T
-    L = MoELayer(lay, max_tokens=T, device=device)
+    # pairs mode: the down GEMM writes bf16 rows, the combine sums them in slot order
+    L = MoELayer(lay, max_tokens=T, device=device, mode=MOE_MODE_PAIRS)
     x = to_device(lay["x"], device)
     del lay
     stream = torch.cuda.Stream(device=device)

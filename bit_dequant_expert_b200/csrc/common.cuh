@@ -12,12 +12,13 @@ constexpr int kWarp = 32;
 
 // ------------------------------------------------------------------ layout
 
-// Workspace header: sticky error word at byte 0, the decode kernel's grid
-// barrier counter at byte 8 (monotonic, 64-bit); the rest of the first 256
-// bytes is reserved.  Scratch sections follow, 256-byte aligned.
+// Workspace header: sticky error word at byte 0, the small-T router's
+// last-block ticket at byte 4 (left at zero by every call), the decode
+// kernel's grid barrier counter at byte 8 (monotonic, 64-bit); the rest of
+// the first 256 bytes is reserved.  Scratch sections follow, 256-byte aligned.
 struct WsHeader {
     int32_t error;
-    int32_t pad;
+    uint32_t route_ticket;
     unsigned long long grid_sync;
     int32_t reserved[60];
 };
@@ -37,16 +38,18 @@ __device__ __forceinline__ float bf16_lo(uint32_t pair) { return __uint_as_float
 __device__ __forceinline__ float bf16_hi(uint32_t pair) { return __uint_as_float(pair & 0xFFFF0000u); }
 __device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_float(uint32_t(b) << 16); }
 
-// fp32 -> bf16 bits, round to nearest even (NaN kept quiet).
+// fp32 -> bf16 bits, round to nearest even (hardware conversion).
 __device__ __forceinline__ uint16_t f32_to_bf16(float f) {
-    uint32_t u = __float_as_uint(f);
-    if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu)) return uint16_t((u >> 16) | 0x40);
-    u += 0x7FFFu + ((u >> 16) & 1u);
-    return uint16_t(u >> 16);
+    uint16_t r;
+    asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(f));
+    return r;
 }
 
+// (lo, hi) -> bf16x2 bits, each rounded to nearest even.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    return uint32_t(f32_to_bf16(lo)) | (uint32_t(f32_to_bf16(hi)) << 16);
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
 }
 
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }

@@ -16,8 +16,9 @@
 //                rows (x rows already gathered into expert order for gate/up,
 //                h rows for down; contiguous either way) into one smem ring
 //                stage; B lands 128B-swizzled and K-major, as the MMA reads it;
-//   warps 2-3    down: each tile's per-column token and routing weight, built
-//                one tile ahead of the epilogue;
+//   warps 2-3    TMA of the B boxes (alternate chunks: one thread keeps only
+//                one box in flight at a time) and, for down, each tile's
+//                per-column token and routing weight for the epilogue;
 //   warps 4-11   dequantise codes to bf16 (scale * q + bias) and write them as
 //                the A operand straight into tensor memory (tcgen05.st), so
 //                the MMA reads only B from shared memory;
@@ -39,9 +40,11 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kNT = 128;                 // token rows per tile (MMA N, max)
+static_assert(kNT % 64 == 0, "the column-table builders cover kNT columns with 64 threads");
 constexpr int kBK = 64;                  // inputs per chunk = one (scale, bias) group
-constexpr int kStages = 8;
-constexpr int kCodesStage = 128 * 32;    // 128 rows x 64 nibbles
+constexpr int kStages = 6;              // B ring and TMEM A stages (64 inputs each)
+constexpr int kCStages = 4;             // codes ring
+constexpr int kCodesStage = 128 * 128;  // 128 rows x 256 nibbles (four chunks), 128B-swizzled
 constexpr int kBStage = kNT * 128;       // kNT rows x 64 bf16
 constexpr int kACol0 = 2 * kNT;          // TMEM: two fp32 accumulators, then the A stages
 constexpr int kAStageCols = kBK / 2;     // bf16 pairs per 32-bit column
@@ -52,9 +55,9 @@ static_assert(kACol0 + kStages * kAStageCols <= kTmemCols, "TMEM budget");
 
 struct Smem {
     uint8_t b[kStages][kBStage];                 // offset 0, 1024-aligned
-    uint8_t codes[kStages][kCodesStage];
+    uint8_t codes[kCStages][kCodesStage];
     uint32_t sbs[2][kSbBytes / 4];               // per-tile (scale, bias) rows, double-buffered
-    uint64_t full[kStages], a_full[kStages], mma_done[kStages];
+    uint64_t full[kStages], a_full[kStages], mma_done[kStages], cfull[kCStages], cempty[kCStages];
     uint64_t acc_full[2], acc_empty[2], tab_full[kTabs], tab_empty[kTabs], sb_full[2], sb_empty[2];
     int tok[kTabs][kNT];
     float w[kTabs][kNT];
@@ -163,6 +166,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int K = gateup ? a.H : a.I;            // reduction length of this GEMM
     const int KC = K / kBK;                      // chunks per tile
     const int ngroups = K / 64;
+    // codes come in stages of cw u32 words (8 cw inputs) per row: 256 inputs,
+    // or all of K when K is shorter; a stage feeds cps chunks
+    const int cw = K >= 256 ? 32 : K / 8;
+    const int cps = cw / 8;
     // (scale, bias) rows go through shared memory by TMA when a row's words
     // span whole 16-byte units; otherwise (tiny K) each thread reads its own
     const bool sb_tma = (ngroups & 3) == 0;
@@ -172,6 +179,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.a_full[s], 8);
             mbar_init(&sm.mma_done[s], 1);
+        }
+        for (int s = 0; s < kCStages; ++s) {
+            mbar_init(&sm.cfull[s], 1);
+            mbar_init(&sm.cempty[s], 8);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.acc_full[b], 1);
@@ -207,31 +218,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
-        // Stage s is refilled once the MMAs of its previous use completed (which
-        // implies its codes were dequantised).  B: one or two 64-row boxes.
-        // The whole next tile's codes and (scale, bias) rows are pulled into L2
-        // while this one streams, so the ring's TMA loads hit L2: a ring of a
-        // few 4 KB stages alone keeps too few bytes in flight for HBM.
-        auto prefetch_tile = [&](int t) {
-            if (t >= ntiles || lane != 0) return;
-            const Tile tl = decode_tile(a, gateup, sm.pre, sm.off, t);
-            const uint8_t* codes = reinterpret_cast<const uint8_t*>(gateup ? a.gu_codes : a.d_codes);
-            const uint8_t* sbb = reinterpret_cast<const uint8_t*>(gateup ? a.gu_sb : a.d_sb);
-            if (gateup) {
-                prefetch_l2(codes + (size_t)wrow_gate(a, tl) * (a.H / 2), 64 * (a.H / 2));
-                prefetch_l2(codes + (size_t)wrow_up(a, tl) * (a.H / 2), 64 * (a.H / 2));
-                prefetch_l2(sbb + (size_t)wrow_gate(a, tl) * (a.H / 16), 64 * (a.H / 16));
-                prefetch_l2(sbb + (size_t)wrow_up(a, tl) * (a.H / 16), 64 * (a.H / 16));
-            } else {
-                prefetch_l2(codes + (size_t)wrow_down(a, tl) * (a.I / 2), 128 * (a.I / 2));
-                prefetch_l2(sbb + (size_t)wrow_down(a, tl) * (a.I / 16), 128 * (a.I / 16));
-            }
-        };
-        prefetch_tile(blockIdx.x);
+        // (scale, bias) rows once per tile, codes once per stage of cps chunks;
+        // a stage is refilled once its chunks were dequantised.
         uint32_t it = 0, lt = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
             const Tile tl = decode_tile(a, gateup, sm.pre, sm.off, t);
-            prefetch_tile(t + gridDim.x);
             if (sb_tma && lane == 0) {
                 const int buf = lt & 1;
                 if (lt >= 2) mbar_wait_bounded(&sm.sb_empty[buf], ((lt >> 1) - 1) & 1, a.err);
@@ -243,20 +234,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_2d(sm.sbs[buf], &sb_map, 0, wrow_down(a, tl), &sm.sb_full[buf]);
                 }
             }
-            const int nbox = tl.npad > 64 ? 2 : 1;
             for (int kc = 0; kc < KC; ++kc, ++it) {
-                const int s = it % kStages;
                 if (lane == 0) {
-                    if (it >= kStages) mbar_wait_bounded(&sm.mma_done[s], ((it / kStages) - 1) & 1, a.err);
-                    mbar_arrive_expect_tx(&sm.full[s], kCodesStage + nbox * 64 * 128);
-                    if (gateup) {
-                        tma_load_2d(sm.codes[s], &codes_map, kc * 8, wrow_gate(a, tl), &sm.full[s]);
-                        tma_load_2d(sm.codes[s] + kCodesStage / 2, &codes_map, kc * 8, wrow_up(a, tl), &sm.full[s]);
-                    } else {
-                        tma_load_2d(sm.codes[s], &codes_map, kc * 8, wrow_down(a, tl), &sm.full[s]);
+                    if (kc % cps == 0) {
+                        const uint32_t cit = it / cps;        // tiles hold whole codes stages
+                        const int cs = cit % kCStages;
+                        if (cit >= kCStages) mbar_wait_bounded(&sm.cempty[cs], ((cit / kCStages) - 1) & 1, a.err);
+                        mbar_arrive_expect_tx(&sm.cfull[cs], 128 * cw * 4);
+                        if (gateup) {
+                            tma_load_2d(sm.codes[cs], &codes_map, kc * 8, wrow_gate(a, tl), &sm.cfull[cs]);
+                            tma_load_2d(sm.codes[cs] + 64 * cw * 4, &codes_map, kc * 8, wrow_up(a, tl), &sm.cfull[cs]);
+                        } else {
+                            tma_load_2d(sm.codes[cs], &codes_map, kc * 8, wrow_down(a, tl), &sm.cfull[cs]);
+                        }
                     }
-                    for (int bx = 0; bx < nbox; ++bx)
-                        tma_load_2d(sm.b[s] + bx * 64 * 128, &b_map, kc * kBK, (int)tl.hrow0 + 64 * bx, &sm.full[s]);
                 }
                 __syncwarp();
             }
@@ -289,16 +280,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else if (warp < 4) {
-        // ------------------------------------------------------------ column tables (down)
-        if (!gateup) {
-            const int bt = tid - 64;
-            uint32_t lt = 0;
-            for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
-                const Tile tl = decode_tile(a, gateup, sm.pre, sm.off, t);
+        // ------------------------------------------------------------ B producers (+ down column tables)
+        // A single thread can keep only one TMA box in flight at a time, so the
+        // B boxes are issued by two warps, alternate chunks each.
+        const int bt = tid - 64;
+        const uint32_t par = warp - 2;
+        uint32_t it = 0, lt = 0;
+        for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
+            const Tile tl = decode_tile(a, gateup, sm.pre, sm.off, t);
+            if (!gateup) {
                 const int slot = lt % kTabs;
                 if (lt >= kTabs) mbar_wait_bounded(&sm.tab_empty[slot], ((lt / kTabs) - 1) & 1, a.err);
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
+                for (int h = 0; h < kNT / 64; ++h) {   // 64 builder threads, kNT columns
                     const int c = bt + 64 * h;
                     int tok = 0;
                     float w = 0.0f;
@@ -322,6 +316,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.tab_full[slot]);
             }
+            const int nbox = tl.npad > 64 ? 2 : 1;   // 64-row boxes
+            for (int kc = 0; kc < KC; ++kc, ++it) {
+                if ((it & 1u) != par) continue;
+                const int s = it % kStages;
+                if (lane == 0) {
+                    if (it >= kStages) mbar_wait_bounded(&sm.mma_done[s], ((it / kStages) - 1) & 1, a.err);
+                    mbar_arrive_expect_tx(&sm.full[s], nbox * 64 * 128);
+                    for (int bx = 0; bx < nbox; ++bx)
+                        tma_load_2d(sm.b[s] + bx * 64 * 128, &b_map, kc * kBK, (int)tl.hrow0 + 64 * bx, &sm.full[s]);
+                }
+                __syncwarp();
+            }
         }
     } else if (warp < 12) {
         // ------------------------------------------------------------ dequantisers
@@ -332,7 +338,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t* sbase = reinterpret_cast<const uint32_t*>(gateup ? a.gu_sb : a.d_sb);
         // codes of row L inside a stage: gate/up interleave gate and up rows on
         // adjacent lanes (even: gate, odd: up), so SwiGLU pairs are lane pairs
-        const int srow_off = gateup ? ((L & 1) * (kCodesStage / 2) + (L >> 1) * 32) : L * 32;
+        // row of lane L inside a codes stage; rows are cw words wide and, when
+        // 128 bytes wide, 128B-swizzled (16-byte unit u of row r sits at u ^ (r & 7))
+        const int crow = gateup ? ((L & 1) * 64 + (L >> 1)) : L;
+        auto codes_at = [&](int cs, int kc) -> uint4 {
+            const int unit = (kc % cps) * 2 + khalf;
+            const int phys = cw == 32 ? (unit ^ (crow & 7)) : unit;
+            return *reinterpret_cast<const uint4*>(sm.codes[cs] + crow * cw * 4 + phys * 16);
+        };
         uint32_t it = 0, lt = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
             const Tile tl = decode_tile(a, gateup, sm.pre, sm.off, t);
@@ -365,13 +378,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kc = 0; kc < KC; kc += 2, it += 2) {
                 const int s0 = it % kStages, s1 = (it + 1) % kStages;
                 const uint32_t sb0 = sb_of(kc), sb1 = sb_of(kc + 1);
-                mbar_wait_bounded(&sm.full[s0], (it / kStages) & 1, a.err);
-                const uint4 cw0 = *reinterpret_cast<const uint4*>(sm.codes[s0] + srow_off + 16 * khalf);
-                mbar_wait_bounded(&sm.full[s1], ((it + 1) / kStages) & 1, a.err);
-                const uint4 cw1 = *reinterpret_cast<const uint4*>(sm.codes[s1] + srow_off + 16 * khalf);
+                const uint32_t cit = it / cps;    // both chunks of the pair share a codes stage (cps even)
+                const int cs = cit % kCStages;
+                mbar_wait_bounded(&sm.cfull[cs], (cit / kCStages) & 1, a.err);
+                const uint4 cw0 = codes_at(cs, kc);
+                const uint4 cw1 = codes_at(cs, kc + 1);
+                if ((kc + 2) % cps == 0) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sm.cempty[cs]);
+                }
                 uint32_t v0[16], v1[16];
                 dequant16(cw0, sb0, v0);
                 dequant16(cw1, sb1, v1);
+                // the MMA reads B from ring stage s0/s1: make sure it landed before
+                // the A operand of the same chunks is declared ready (the MMA
+                // also waits on it, this keeps the two rings in step)
                 if (it >= kStages) mbar_wait_bounded(&sm.mma_done[s0], ((it / kStages) - 1) & 1, a.err);
                 if (it + 1 >= kStages) mbar_wait_bounded(&sm.mma_done[s1], (((it + 1) / kStages) - 1) & 1, a.err);
                 tc_fence_after();
@@ -480,13 +501,14 @@ EncodeTiled encode_fn() {
 bool make_codes_map(CUtensorMap* m, const uint32_t* codes, int rows, int K, int box_rows) {
     EncodeTiled enc = encode_fn();
     if (!enc) return false;
+    const int cw = K >= 256 ? 32 : K / 8;      // words per row per box, as the kernel reads them
     const cuuint64_t dims[2] = {(cuuint64_t)(K / 8), (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-    const cuuint32_t box[2] = {8, (cuuint32_t)box_rows};
+    const cuuint32_t box[2] = {(cuuint32_t)cw, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(codes), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+               CU_TENSOR_MAP_INTERLEAVE_NONE, cw == 32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // bf16 [rows, cols] activations read in boxes of 64 columns (128 bytes) x

@@ -19,6 +19,7 @@ struct RouterArgs {
     float* topk_w;
     int32_t* counts;
     float* logits_ws;   // [T, E] scratch
+    uint32_t* ticket;   // last-block ticket of the small-T router (workspace header, zero between calls)
     int32_t* err;
 };
 

@@ -113,6 +113,7 @@ int32_t moe_route(const moe_config_t* cfg, int32_t T, const uint16_t* x, const u
     a.topk_w = topk_w;
     a.counts = counts;
     a.logits_ws = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + layout(cfg, T).logits);
+    a.ticket = &reinterpret_cast<WsHeader*>(ws)->route_ticket;
     a.err = err_word(ws);
     return cuda_status(launch_router(a, (cudaStream_t)stream));
 }
@@ -245,7 +246,7 @@ int32_t moe_get_device_error(const void* ws, void* stream) {
 int32_t moe_launch_count(const moe_config_t* cfg, int32_t T, int32_t mode, int32_t path) {
     if (!config_ok(cfg) || T < 1 || T > kMaxTokens) return -1;
     if (mode != MOE_MODE_SCATTER && mode != MOE_MODE_PAIRS) return -1;
-    const int route = 2;
+    const int route = T <= 8 ? 1 : 2;
     const int permute = T <= 256 ? 1 : 3;
     const FfnArgs a = shape_only(cfg, T);
     if (path == MOE_PATH_AUTO) path = resolve_path(a);

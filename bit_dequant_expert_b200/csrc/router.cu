@@ -17,14 +17,10 @@ namespace moe {
 // exactly like the contract); the 32 lane partials are then combined by the
 // xor butterfly 16, 8, 4, 2, 1.  A block has 8 warps stacked along experts.
 template <int TT, int TE>
-__global__ void __launch_bounds__(256) k_router_logits(int T, int H, int E, const uint16_t* __restrict__ x,
-                                                       const uint16_t* __restrict__ wr,
-                                                       const float* __restrict__ bias, int64_t bias_stride,
-                                                       float* __restrict__ logits) {
+__device__ __forceinline__ void router_tile(int T, int H, int E, int t0, int e0, const uint16_t* __restrict__ x,
+                                            const uint16_t* __restrict__ wr, const float* __restrict__ bias,
+                                            int64_t bias_stride, float* __restrict__ logits) {
     const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int t0 = blockIdx.x * TT;
-    const int e0 = (blockIdx.y * 8 + warp) * TE;
     if (e0 >= E) return;
     const int nchunk = H / 8;
 
@@ -35,25 +31,34 @@ __global__ void __launch_bounds__(256) k_router_logits(int T, int H, int E, cons
         for (int b = 0; b < TE; ++b) acc[a][b] = 0.0f;
 
     for (int c = lane; c < nchunk; c += 32) {
-        uint4 xv[TT];
+        // this chunk of every token, widened to fp32 once and reused for all TE experts
+        float xf[TT][8];
 #pragma unroll
         for (int a = 0; a < TT; ++a) {
             const int t = t0 + a;
-            xv[a] = (t < T) ? *reinterpret_cast<const uint4*>(x + (size_t)t * H + 8 * c) : make_uint4(0, 0, 0, 0);
+            const uint4 xv = (t < T) ? *reinterpret_cast<const uint4*>(x + (size_t)t * H + 8 * c) : make_uint4(0, 0, 0, 0);
+            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                xf[a][2 * q] = bf16_lo(xw[q]);
+                xf[a][2 * q + 1] = bf16_hi(xw[q]);
+            }
         }
 #pragma unroll
         for (int b = 0; b < TE; ++b) {
             const uint4 wv = *reinterpret_cast<const uint4*>(wr + (size_t)(e0 + b) * H + 8 * c);
             const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+            float wf[8];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                wf[2 * q] = bf16_lo(ww[q]);
+                wf[2 * q + 1] = bf16_hi(ww[q]);
+            }
 #pragma unroll
             for (int a = 0; a < TT; ++a) {
-                const uint32_t xw[4] = {xv[a].x, xv[a].y, xv[a].z, xv[a].w};
                 float s = acc[a][b];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    s = __fmaf_rn(bf16_lo(xw[q]), bf16_lo(ww[q]), s);
-                    s = __fmaf_rn(bf16_hi(xw[q]), bf16_hi(ww[q]), s);
-                }
+                for (int j = 0; j < 8; ++j) s = __fmaf_rn(xf[a][j], wf[j], s);   // inputs ascending in the chunk
                 acc[a][b] = s;
             }
         }
@@ -81,6 +86,18 @@ __global__ void __launch_bounds__(256) k_router_logits(int T, int H, int E, cons
     }
 }
 
+template <int TT, int TE>
+__global__ void __launch_bounds__(256) k_router_logits(int T, int H, int E, const uint16_t* __restrict__ x,
+                                                       const uint16_t* __restrict__ wr,
+                                                       const float* __restrict__ bias, int64_t bias_stride,
+                                                       float* __restrict__ logits, int32_t* __restrict__ counts) {
+    // the top-k kernel that follows on the stream accumulates the counts
+    if (counts && blockIdx.x == 0 && blockIdx.y == 0)
+        for (int e = threadIdx.x; e < E; e += blockDim.x) counts[e] = 0;
+    const int warp = threadIdx.x >> 5;
+    router_tile<TT, TE>(T, H, E, blockIdx.x * TT, (blockIdx.y * 8 + warp) * TE, x, wr, bias, bias_stride, logits);
+}
+
 // Order-preserving map of a finite float to uint32 (larger float -> larger
 // key); -0.0 is folded onto +0.0 so the two tie.
 __device__ __forceinline__ uint32_t order_key(float f) {
@@ -98,19 +115,17 @@ __device__ __forceinline__ float key_value(uint32_t k) {
 // the winner.  Weights are the softmax over the K selected logits, which is
 // the E-way softmax restricted to them and renormalised.
 template <int EPL, int K>
-__global__ void __launch_bounds__(256) k_topk(int T, int E, const float* __restrict__ logits,
-                                              const float* __restrict__ bias, int64_t bias_stride,
-                                              int32_t* __restrict__ idx, float* __restrict__ wout,
-                                              int32_t* __restrict__ counts, int32_t* err) {
+__device__ __forceinline__ void topk_token(int t, int E, const float* __restrict__ logits,
+                                           const float* __restrict__ bias, int64_t bias_stride,
+                                           int32_t* __restrict__ idx, float* __restrict__ wout,
+                                           int32_t* __restrict__ counts, int32_t* err) {
     const int lane = threadIdx.x & 31;
-    const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (t >= T) return;
     float v[EPL];
     bool bad = false;
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
         const int e = lane + 32 * i;
-        float l = logits[(size_t)t * E + e];
+        float l = __ldcg(logits + (size_t)t * E + e);
         if (bias) l = __fadd_rn(l, bias[(int64_t)t * bias_stride + e]);
         v[i] = l;
         bad |= !isfinite(l);
@@ -167,23 +182,58 @@ __global__ void __launch_bounds__(256) k_topk(int T, int E, const float* __restr
     }
 }
 
+template <int EPL, int K>
+__global__ void __launch_bounds__(256) k_topk(int T, int E, const float* __restrict__ logits,
+                                              const float* __restrict__ bias, int64_t bias_stride,
+                                              int32_t* __restrict__ idx, float* __restrict__ wout,
+                                              int32_t* __restrict__ counts, int32_t* err) {
+    const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (t >= T) return;
+    topk_token<EPL, K>(t, E, logits, bias, bias_stride, idx, wout, counts, err);
+}
+
+// A handful of tokens (T <= 8) in one launch: every block computes the logits
+// of all tokens for 8 experts (one per warp); the last block to finish (an
+// atomic ticket, reset by that block for the next call) selects the top-k of
+// every token and writes the counts.
+__global__ void __launch_bounds__(256) k_route_small(int T, int H, int E, const uint16_t* __restrict__ x,
+                                                     const uint16_t* __restrict__ wr,
+                                                     const float* __restrict__ bias, int64_t bias_stride,
+                                                     float* __restrict__ logits, int32_t* __restrict__ idx,
+                                                     float* __restrict__ wout, int32_t* __restrict__ counts,
+                                                     uint32_t* ticket, int32_t* err) {
+    __shared__ bool last;
+    const int warp = threadIdx.x >> 5;
+    router_tile<8, 1>(T, H, E, 0, blockIdx.x * 8 + warp, x, wr, bias, bias_stride, logits);
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) last = atomicAdd(ticket, 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) counts[e] = 0;
+    __syncthreads();
+    if (warp < T) topk_token<8, 8>(warp, E, logits, nullptr, 0, idx, wout, counts, err);
+    if (threadIdx.x == 0) *ticket = 0u;
+}
+
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t st) {
-    cudaError_t ce = cudaMemsetAsync(a.counts, 0, sizeof(int32_t) * a.E, st);
-    if (ce != cudaSuccess) return ce;
+    if (!a.logits_in && a.T <= 8 && a.E == 256) {
+        k_route_small<<<a.E / 8, 256, 0, st>>>(a.T, a.H, a.E, a.x, a.w_router, a.bias, a.bias_stride, a.logits_ws,
+                                               a.topk_idx, a.topk_w, a.counts, a.ticket, a.err);
+        return cudaGetLastError();
+    }
     const float* lg = a.logits_in;
     const float* topk_bias = a.bias;
     if (!lg) {
-        if (a.T <= 4) {
-            dim3 grid(a.T, a.E / 8);
-            k_router_logits<1, 1><<<grid, 256, 0, st>>>(a.T, a.H, a.E, a.x, a.w_router, a.bias, a.bias_stride,
-                                                         a.logits_ws);
-        } else {
-            dim3 grid((a.T + 7) / 8, a.E / 64);
-            k_router_logits<8, 8><<<grid, 256, 0, st>>>(a.T, a.H, a.E, a.x, a.w_router, a.bias, a.bias_stride,
-                                                         a.logits_ws);
-        }
+        dim3 grid((a.T + 7) / 8, a.E / 64);
+        k_router_logits<8, 8><<<grid, 256, 0, st>>>(a.T, a.H, a.E, a.x, a.w_router, a.bias, a.bias_stride,
+                                                     a.logits_ws, a.counts);
         lg = a.logits_ws;
         topk_bias = nullptr;
+    } else {
+        cudaError_t ce = cudaMemsetAsync(a.counts, 0, sizeof(int32_t) * a.E, st);
+        if (ce != cudaSuccess) return ce;
     }
     k_topk<8, 8><<<(a.T + 7) / 8, 256, 0, st>>>(a.T, a.E, lg, topk_bias, a.bias_stride, a.topk_idx, a.topk_w,
                                                 a.counts, a.err);
