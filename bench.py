@@ -361,6 +361,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-prefill", action="store_true", help="skip the T=2048 prefill measurement")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="measure only the T=2048 prefill layer (its line replaces the decode line)")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle CPU baseline")
     args = ap.parse_args(argv)
     warmup = max(args.warmup, 3)
@@ -377,6 +379,26 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     device = torch.device("cuda", torch.cuda.current_device())
     peaks = load_peaks()
+
+    if args.prefill_only:
+        pre = run_prefill(device, max(args.steps, 1), warmup, world, peaks)
+        ms, units = aggregate(pre["ms_per_step"], 2048, world)
+        line = {"metric": "MoE expert-layer tokens/s (T=2048 prefill layer)", "value": units / (ms / 1e3),
+                "unit": UNIT, "n_gpus": world, "steps": pre["steps"], "warmup": warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16 (4-bit weights, fp32 accumulation)",
+                "data": "synthetic (seeded; SplitMix64 layers shaped like the pages' model)",
+                "config": {"workload": pre["workload"], "global_batch": 2048 * world, "seq_len": 2048,
+                           "parallelism": "replicas" if world > 1 else "single GPU", "l2": pre["l2"]},
+                "roofline": pre["roofline"], "gpu_launches": pre["gpu_launches_per_step"] * pre["steps"],
+                "breakdown_us": pre["breakdown_us"], "peaks": peaks}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            barrier(world)
+            dist.destroy_process_group()
+        return 0
 
     res = run_decode(device, args.steps, warmup, world, peaks)
     pre = None if args.no_prefill else run_prefill(device, max(args.steps // 10, 5), warmup, world, peaks)

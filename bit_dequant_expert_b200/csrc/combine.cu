@@ -4,12 +4,15 @@
 // second paragraph (eight routed experts plus one shared expert per token).
 #include "common.cuh"
 #include "kernels.h"
+#include "ptx.cuh"
 
 namespace moe {
 
 // y = bf16(y_acc), eight values per thread.
 __global__ void __launch_bounds__(256) k_combine_scatter(size_t n8, const float* __restrict__ y_acc,
                                                          uint16_t* __restrict__ y) {
+    griddep_wait();   // y_acc comes from the expert FFN
+    griddep_launch_dependents();
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8; i += (size_t)gridDim.x * blockDim.x) {
         const float4 a = reinterpret_cast<const float4*>(y_acc)[2 * i];
         const float4 b = reinterpret_cast<const float4*>(y_acc)[2 * i + 1];
@@ -33,6 +36,8 @@ __global__ void __launch_bounds__(256) k_combine_pairs(int T, int H, int has_sha
     const int t = blockIdx.x;
     __shared__ int s_row[K];
     __shared__ float s_w[K];
+    griddep_wait();   // rows come from the expert FFN
+    griddep_launch_dependents();
     if (threadIdx.x < K) {
         int r = pair_to_row[(size_t)t * K + threadIdx.x];
         if (r < 0 || r >= T * K) {
@@ -79,12 +84,10 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st) {
     if (a.mode == MOE_MODE_SCATTER) {
         const size_t n8 = (size_t)a.T * a.H / 8;
         const int blocks = (int)std::min<size_t>((n8 + 255) / 256, 148 * 16);
-        k_combine_scatter<<<blocks, 256, 0, st>>>(n8, a.y_acc, a.y);
-    } else {
-        k_combine_pairs<8><<<a.T, 256, 0, st>>>(a.T, a.H, a.has_shared, a.rows, a.shared, a.pair_to_row, a.w, a.y,
-                                               a.err);
+        return launch_pdl(k_combine_scatter, dim3(blocks), dim3(256), 0, st, n8, a.y_acc, a.y);
     }
-    return cudaGetLastError();
+    return launch_pdl(k_combine_pairs<8>, dim3(a.T), dim3(256), 0, st, a.T, a.H, a.has_shared, a.rows, a.shared,
+                      a.pair_to_row, a.w, a.y, a.err);
 }
 
 }  // namespace moe

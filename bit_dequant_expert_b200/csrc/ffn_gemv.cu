@@ -1,5 +1,5 @@
-// Expert FFNs for a handful of tokens (T <= 8, decode): one persistent,
-// cooperative kernel per call, bound by HBM bandwidth.
+// Expert FFNs for a handful of tokens (T <= 8, decode): one kernel per call,
+// bound by HBM bandwidth.
 //
 // Lily pages: "Perplexity's Lily brings fast local AI to Apple silicon Macs",
 // section "Where the Engine Gains Speed" (decode minimises the bytes moved per
@@ -8,26 +8,36 @@
 // Argument" (decode has little reuse, so memory traffic dominates).
 //
 // Design (B200):
-//  - One CTA per SM.  Warp 16 is a producer: it streams the packed rows of
-//    every active expert (codes and (scale, bias) rows, exactly the bytes of
-//    the active experts, each once) into a ring of shared-memory stages with
-//    1-D bulk async copies completing on mbarriers.  Warps 0..15 consume the
-//    ring as four quads.
-//  - Consumers turn 4-bit codes into bf16 weights in registers (byte permute,
-//    mask, one bf16x2 subtract and one bf16x2 fma per two weights) laid out
-//    as warp-MMA A fragments; the tokens are the MMA's N = 8 columns, so up
-//    to 8 tokens cost the same as one.  The k order inside a 128-input step
-//    is permuted identically on both operands (ldmatrix hands each lane one
-//    code word of four consecutive 16-byte chunks), which a dot product does
-//    not see.
-//  - Phase 1: gate/up rows of 8 outputs (gate j0..j0+7 on MMA rows 0..7, up
-//    j0..j0+7 on rows 8..15, so SwiGLU pairs sit in one thread), K split over
-//    the quad's four warps and reduced in shared memory; h is stored in bf16.
-//  - A bounded grid barrier (every CTA is co-resident: cooperative launch)
-//    separates phase 1 from phase 2; the producer keeps prefetching phase-2
-//    (down) weights across it.
-//  - Phase 2: 64 down rows per stage, 16 per warp, full K; the epilogue adds
-//    w * y into y_acc (scatter mode, zeroed in phase 1) or stores bf16 rows.
+//  - Work unit = (active expert, 32-wide block of the intermediate size); at
+//    T = 1 the 9 experts x 16 blocks fill 144 of the 148 SMs, one CTA each.
+//    A CTA computes gate/up + SwiGLU for its 32 intermediate columns over all
+//    of H, keeps those 32 h values in shared memory, and multiplies them by
+//    the matching 32 columns of the down matrix for every output row
+//    (split-K over the intermediate size), adding w * y into y_acc.  No CTA
+//    waits for another.
+//  - A producer warp moves each unit in a few large TMA boxes: gate and up
+//    codes of 8 of the 32 rows per box, whole rows (16 KB: two contiguous
+//    8 KB runs of HBM; 128B-swizzled so the consumers' 16-byte reads hit
+//    distinct banks), and
+//    the block's down codes (H rows x 16 B, one box).  The shared expert's
+//    units do not depend on routing, so their loads are issued before the
+//    kernel waits on the previous grid (programmatic dependent launch).
+//  - Consumers (16 warps) turn 4-bit codes into bf16 weights in registers
+//    (shift, one mask-or, one bf16x2 subtract and one bf16x2 fma per two
+//    weights) laid out as warp-MMA A fragments; tokens are the MMA's N = 8
+//    columns.  A code word yields the nibble pairs (j, j+4); x and h are kept
+//    in shared memory in the same order inside every 8-element group, so the
+//    dot products see matching operands.  Box t feeds row tile t (four
+//    warps, one quarter of H each), so work starts with the first box to
+//    land.  (scale, bias) words come straight from global memory into
+//    registers at the start of a unit.
+//  - y_acc is zeroed by the kernel itself: every CTA clears a slice and
+//    counts itself in a monotonic counter; the producer warp waits for the
+//    full count while the consumers compute, and the first accumulation
+//    waits on its signal.  All CTAs are co-resident (one per SM), and every
+//    wait is bounded.
+#include <cuda.h>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
@@ -40,244 +50,177 @@ constexpr int kConsumerWarps = 16;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMaxT = 8;
 constexpr int kMaxActive = 257;
-constexpr int kMaxStages = 8;
-constexpr int kSmemBudget = 225 * 1024;
+constexpr int kCodeSlots = 4;
+constexpr int kCodePiece = 2 * 8 * 8 * 128;    // (gate, up) x 8 chunks x 8 rows x 128 B
+constexpr int kJ = 32;                           // intermediate columns per unit
 
 struct GemvLayout {
-    int rs1, rs2;        // code-row strides in a stage (bytes), phase 1 / phase 2
-    int stage_bytes;     // one ring stage
-    int stages;          // ring depth
-    int xs;              // padded x row stride (bytes)
-    int hs;              // padded h row stride (bytes) of the phase-2 staging
-    int off_ring, off_x, off_red, off_tab, off_bar, total;
+    int d_piece;   // H rows x 16 B
+    int xs;        // x row stride (bytes)
+    int off_code, off_d, off_x, off_red, off_h, off_dsb, off_tab, off_bar, total;
 };
 
 __host__ __device__ inline int round_up(int v, int a) { return (v + a - 1) / a * a; }
 
-__host__ __device__ inline GemvLayout gemv_layout(int H, int I) {
+__host__ __device__ inline GemvLayout gemv_layout(int H) {
     GemvLayout L;
-    L.rs1 = H / 2;
-    L.rs2 = I / 2;
-    const int p1 = 16 * L.rs1 + 16 * (H / 16);
-    const int p2 = 64 * L.rs2 + 64 * (I / 16);
-    L.stage_bytes = round_up(p1 > p2 ? p1 : p2, 128);
+    L.d_piece = H * 16;
     L.xs = 2 * H + 16;
-    L.hs = 2 * I + 16;
-    // phase 1 reads the x tile, phase 2 reuses the same bytes for each quad's h rows
-    const int x_need = kMaxT * L.xs, h_need = 4 * kMaxT * L.hs;
-    const int x_bytes = round_up(x_need > h_need ? x_need : h_need, 128);
-    const int red_bytes = 4 * 4 * 32 * 16;
-    // act_e, act_row0, act_cnt, then per (active, i): token, weight
-    const int tab_bytes = round_up(kMaxActive * 3 * 4 + kMaxActive * kMaxT * 8 + 64, 128);
-    const int bar_bytes = 2 * kMaxStages * 8;
-    const int fixed = x_bytes + red_bytes + tab_bytes + bar_bytes + 1024;
-    int s = (kSmemBudget - fixed) / L.stage_bytes;
-    L.stages = s > kMaxStages ? kMaxStages : s;
-    L.off_ring = 0;
-    L.off_x = L.stages * L.stage_bytes;
-    L.off_red = L.off_x + x_bytes;
-    L.off_tab = L.off_red + red_bytes;
-    L.off_bar = L.off_tab + tab_bytes;
-    L.total = L.off_bar + bar_bytes;
+    L.off_code = 0;
+    L.off_d = L.off_code + kCodeSlots * kCodePiece;
+    L.off_x = round_up(L.off_d + 2 * L.d_piece, 1024);
+    L.off_red = round_up(L.off_x + kMaxT * L.xs, 128);
+    L.off_h = L.off_red + kConsumerWarps * 32 * 16;
+    L.off_dsb = round_up(L.off_h + 2 * kMaxT * kJ * 2, 128);   // [2][H] down (scale, bias) words
+    L.off_tab = L.off_dsb + 2 * H * 4;
+    // act_e, act_row0, act_cnt [kMaxActive]; row -> pair [64]; pair -> weight [64]; misc [4]
+    L.off_bar = round_up(L.off_tab + (3 * kMaxActive + 64 + 64 + 4) * 4, 128);
+    L.total = L.off_bar + 32 * 8;
     return L;
 }
 
 struct GemvArgs {
     FfnArgs f;
     GemvLayout L;
-    unsigned long long* sync;   // grid barrier arrival counter (monotonic)
+    unsigned long long* sync;   // monotonic arrival counter (workspace header)
 };
 
-// Per-CTA schedule: phase-1 tiles v = b, b+G, ... < V1, then phase-2 stages.
-struct Sched {
-    int b, G, V1, V2, n1, n2;
-    __device__ void init(int A, int I, int H) {
-        b = blockIdx.x;
-        G = gridDim.x;
-        V1 = A * (I / 8);
-        V2 = A * (H / 64);
-        n1 = b < V1 ? (V1 - b + G - 1) / G : 0;
-        n2 = b < V2 ? (V2 - b + G - 1) / G : 0;
-    }
-    __device__ int total() const { return n1 + n2; }
-    __device__ bool phase1(int l) const { return l < n1; }
-    __device__ int unit(int l) const { return l < n1 ? b + l * G : b + (l - n1) * G; }
-};
-
-__device__ __forceinline__ uint32_t dup_lo(uint32_t w) { return prmt(w, w, 0x1010); }
-__device__ __forceinline__ uint32_t dup_hi(uint32_t w) { return prmt(w, w, 0x3232); }
-
-// 16 x 8 x (128 * nsteps) MMA over a stage's code rows [0, 16) (row stride
-// rs bytes, 64 bytes of codes per 128-input step).  Lane (g, c) = (lane/4,
-// lane%4) reads the 16-byte chunk c of rows g and g+8, i.e. inputs
-// [32c, 32c+32) of the step, which lie in one (scale, bias) group.  Within a
-// step, MMA k-step (w, half) takes the inputs 32c + 8w + 4half + {0..3} of
-// every c: the two operands are permuted alike, which a dot product does not
-// see.  B fragments come from bsrc(S, w): 8 bf16 of the lane's column g at
-// inputs 128S + 32c + 8w.  (scale, bias) rows hold `ngroups` u32 each.
-template <typename BLoad>
-__device__ __forceinline__ void mma_rows16(float (&acc)[4], const uint8_t* codes, int rs, const uint32_t* sb,
-                                           int ngroups, int step0, int nsteps, BLoad bsrc) {
-    const int lane = threadIdx.x & 31;
-    const int g = lane >> 2, c = lane & 3;
-    const uint8_t* rowA = codes + (size_t)g * rs + 16 * c;
-    const uint8_t* rowB = rowA + 8 * rs;
-    float part[4][4];   // one accumulator chain per code word: four independent MMA chains
-#pragma unroll
-    for (int w = 0; w < 4; ++w)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) part[w][q] = 0.0f;
-    for (int S = step0; S < step0 + nsteps; ++S) {
-        const uint4 ca = *reinterpret_cast<const uint4*>(rowA + S * 64);
-        const uint4 cb = *reinterpret_cast<const uint4*>(rowB + S * 64);
-        const int grp = 2 * S + (c >> 1);
-        const uint32_t swA = sb[(size_t)g * ngroups + grp];
-        const uint32_t swB = sb[(size_t)(g + 8) * ngroups + grp];
-        const uint32_t sA = dup_lo(swA), bA = dup_hi(swA), sB = dup_lo(swB), bB = dup_hi(swB);
-        const uint32_t wa[4] = {ca.x, ca.y, ca.z, ca.w};
-        const uint32_t wb[4] = {cb.x, cb.y, cb.z, cb.w};
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            const uint4 xv = bsrc(S, w);
-            const uint32_t vA = wa[w], vA4 = vA >> 4, vB = wb[w], vB4 = vB >> 4;
-            mma_bf16_16816(part[w], dequant_pair<0>(vA, vA4, sA, bA), dequant_pair<0>(vB, vB4, sB, bB),
-                           dequant_pair<1>(vA, vA4, sA, bA), dequant_pair<1>(vB, vB4, sB, bB), xv.x, xv.y);
-            mma_bf16_16816(part[w], dequant_pair<2>(vA, vA4, sA, bA), dequant_pair<2>(vB, vB4, sB, bB),
-                           dequant_pair<3>(vA, vA4, sA, bA), dequant_pair<3>(vB, vB4, sB, bB), xv.z, xv.w);
-        }
-    }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) acc[q] += (part[0][q] + part[1][q]) + (part[2][q] + part[3][q]);
-}
-
-__device__ __forceinline__ uint4 ld_cg_v4(const void* p) {
-    uint4 v;
-    asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
-
-// Bounded grid-wide barrier over all CTAs of a cooperative launch.  The
-// counter only ever grows: a launch whose CTAs read `base` at start (a
-// multiple of the grid size, since every earlier launch completed) is
-// released when the counter reaches base + gridDim.x.
 __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
     unsigned long long v;
     asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
 }
 
-__device__ void grid_barrier(unsigned long long* counter, unsigned long long target, int32_t* err) {
-    __threadfence();
-    atomicAdd(counter, 1ull);
-    const uint64_t t0 = globaltimer_ns();
-    while (ld_acquire_u64(counter) < target) {
-        if (globaltimer_ns() - t0 > 500000000ull) {
-            set_error(err, MOE_ERR_TIMEOUT);
-            break;
-        }
-    }
-    __threadfence();
+__device__ __forceinline__ unsigned long long atom_add_release_u64(unsigned long long* p, unsigned long long v) {
+    unsigned long long old;
+    asm volatile("atom.add.release.gpu.global.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
+    return old;
 }
 
-__global__ void __launch_bounds__(kThreads, 1) k_ffn_gemv(GemvArgs ga) {
-    extern __shared__ __align__(1024) uint8_t smem[];
+// MMA row g of a gate/up tile <-> row 8t + perm8(g) of the unit's 32: rows read
+// by one 8-lane phase then differ in bit 2 of (row & 7), which the 128-byte
+// swizzle turns into distinct banks.
+__device__ __forceinline__ int perm8(int g) { return (g >> 1) | ((g & 1) << 2); }
+
+// Position of element i of an 8-group in the split order (0,4,1,5,2,6,3,7).
+__device__ __forceinline__ int split_pos(int i) { return i < 4 ? 2 * i : 2 * (i - 4) + 1; }
+
+// 8 consecutive bf16 (as 4 pairs) -> the split order.
+__device__ __forceinline__ uint4 to_split_order(uint4 v) {
+    uint4 r;
+    r.x = prmt(v.x, v.z, 0x5410);
+    r.y = prmt(v.x, v.z, 0x7632);
+    r.z = prmt(v.y, v.w, 0x5410);
+    r.w = prmt(v.y, v.w, 0x7632);
+    return r;
+}
+
+// Two MMAs over one code word per row: rows g / g+8 give words va / vb, the
+// (scale, bias) pairs s/b, the B fragment pairs bx (split order).
+__device__ __forceinline__ void mma_word(float (&d)[4], uint32_t va, uint32_t vb, uint32_t sA, uint32_t bA,
+                                         uint32_t sB, uint32_t bB, uint4 bx) {
+    mma_bf16_16816(d, dequant_split(va, sA, bA), dequant_split(vb, sB, bB), dequant_split(va >> 4, sA, bA),
+                   dequant_split(vb >> 4, sB, bB), bx.x, bx.y);
+    mma_bf16_16816(d, dequant_split(va >> 8, sA, bA), dequant_split(vb >> 8, sB, bB),
+                   dequant_split(va >> 12, sA, bA), dequant_split(vb >> 12, sB, bB), bx.z, bx.w);
+}
+
+__device__ __forceinline__ uint32_t sb_scale2(uint32_t w) { return prmt(w, w, 0x1010); }
+__device__ __forceinline__ uint32_t sb_bias2(uint32_t w) { return prmt(w, w, 0x3232); }
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_ffn_gemv(const __grid_constant__ CUtensorMap gu_map, const __grid_constant__ CUtensorMap d_map,
+               const GemvArgs ga) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const FfnArgs& a = ga.f;
     const GemvLayout& L = ga.L;
     const int H = a.H, I = a.I, E = a.E, K = a.K, T = a.T;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int NJ = I / kJ;          // units per expert
+    const int NP = H / 512;         // 128-input steps per warp (a quarter of H)
+    const int NCH = H / 256;        // 256-input chunks (128-byte lines) per gate/up row
+    const int ngr = H / 64;         // (scale, bias) groups per gate/up row
+    const int NB = I / 64;          // (scale, bias) groups per down row
 
     int* act_e = reinterpret_cast<int*>(smem + L.off_tab);
     int* act_row0 = act_e + kMaxActive;
     int* act_cnt = act_row0 + kMaxActive;
-    int* act_tok = act_cnt + kMaxActive;                       // [kMaxActive][kMaxT]
-    float* act_w = reinterpret_cast<float*>(act_tok + kMaxActive * kMaxT);
-    int* s_misc = reinterpret_cast<int*>(act_w + kMaxActive * kMaxT);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.off_bar);
-    uint64_t* empty = full + kMaxStages;
-    uint8_t* xs = smem + L.off_x;
+    int* s_r2p = act_cnt + kMaxActive;
+    float* s_pw = reinterpret_cast<float*>(s_r2p + 64);
+    int* s_misc = reinterpret_cast<int*>(s_pw + 64);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.off_bar);
+    uint64_t* code_full = bars;
+    uint64_t* code_empty = bars + 4;
+    uint64_t* d_full = bars + 8;
+    uint64_t* d_empty = bars + 10;
+    uint64_t* zero_done = bars + 12;   // every CTA has cleared its slice of y_acc
+    uint16_t* hbuf = reinterpret_cast<uint16_t*>(smem + L.off_h);   // [2][kMaxT][kJ], split order
     float4* red = reinterpret_cast<float4*>(smem + L.off_red);
+    uint8_t* xs = smem + L.off_x;                                    // [kMaxT][H], split order
+    uint32_t* dsb_s = reinterpret_cast<uint32_t*>(smem + L.off_dsb);  // [2][H]
 
+    if (warp == kConsumerWarps && lane == 0) {
+        prefetch_tensormap(&gu_map);
+        prefetch_tensormap(&d_map);
+    }
     if (tid == 0) {
-        for (int st = 0; st < L.stages; ++st) {
-            mbar_init(&full[st], 1);
-            mbar_init(&empty[st], 4);
+        for (int i = 0; i < kCodeSlots; ++i) {
+            mbar_init(&code_full[i], 1);
+            mbar_init(&code_empty[i], 4);   // the box's row tile: four warps
         }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&d_full[i], 1);
+            mbar_init(&d_empty[i], kConsumerWarps);
+        }
+        mbar_init(zero_done, 1);
         fence_mbar_init();
     }
     __syncthreads();
 
-    // Phase-1 units: v = a * (I/8) + jt over the active experts, the shared
-    // expert first (a = 0).  Unit b of this CTA is then known before any
-    // routing output is read: the shared expert's tile b, if b < I/8.
-    auto issue_phase1 = [&](int slot, int e, int j0) {
-        // gate rows j0..j0+7 and up rows I+j0..I+j0+7 are contiguous in memory:
-        // two copies of codes, two of (scale, bias)
-        uint8_t* st = smem + L.off_ring + (size_t)slot * L.stage_bytes;
-        const uint8_t* codes = reinterpret_cast<const uint8_t*>(a.gu_codes) + (size_t)e * 2 * I * (H / 2);
-        const uint8_t* sbg = reinterpret_cast<const uint8_t*>(a.gu_sb) + (size_t)e * 2 * I * (H / 16);
-        if (lane == 0) {
-            mbar_arrive_expect_tx(&full[slot], 16 * (H / 2) + 16 * (H / 16));
-            bulk_g2s(st, codes + (size_t)j0 * (H / 2), 8 * (H / 2), &full[slot]);
-            bulk_g2s(st + 8 * (H / 2), codes + (size_t)(I + j0) * (H / 2), 8 * (H / 2), &full[slot]);
-            bulk_g2s(st + 16 * (H / 2), sbg + (size_t)j0 * (H / 16), 8 * (H / 16), &full[slot]);
-            bulk_g2s(st + 16 * (H / 2) + 8 * (H / 16), sbg + (size_t)(I + j0) * (H / 16), 8 * (H / 16), &full[slot]);
+    // Loads of unit k of this CTA (expert e, column block jb); producer lane 0.
+    auto issue_unit = [&](int k, int e, int jb) {
+        for (int p = 0; p < 4; ++p) {
+            const int n = k * 4 + p, cs = n % kCodeSlots;
+            if (n >= kCodeSlots) mbar_wait_bounded(&code_empty[cs], ((n / kCodeSlots) - 1) & 1, a.err);
+            mbar_arrive_expect_tx(&code_full[cs], 2 * 8 * (H / 2));   // 8 gate + 8 up rows of H/2 bytes
+            tma_load_5d(smem + L.off_code + cs * kCodePiece, &gu_map, 0, kJ * jb + 8 * p, 0, 0, e, &code_full[cs]);
         }
-        __syncwarp();
+        const int ds = k & 1;
+        if (k >= 2) mbar_wait_bounded(&d_empty[ds], ((k >> 1) - 1) & 1, a.err);
+        mbar_arrive_expect_tx(&d_full[ds], L.d_piece);
+        tma_load_4d(smem + L.off_d + ds * L.d_piece, &d_map, 0, 0, e * (H / 256), jb, &d_full[ds]);
     };
-    const bool early = a.has_shared && (int)blockIdx.x < I / 8;
-    if (warp == kConsumerWarps && early) issue_phase1(0, E, blockIdx.x * 8);
-    // Work that needs no routing output: the x tile (tokens on the MMA's 8
-    // columns, zero beyond T), zeroing this CTA's slice of y_acc, and the
-    // grid-barrier base.
-    unsigned long long bar_base = 0;
-    int r2p = 0;
-    float pw = 0.0f;
-    if (tid < T * K) {      // T <= 8: every (row -> pair) entry and routing weight, loaded up front
-        r2p = a.row_to_pair[tid];
-        pw = a.topk_w[tid];
-    }
-    if (warp < kConsumerWarps) {
-        for (int q = tid; q < kMaxT * (H / 8); q += kConsumerWarps * 32) {
-            const int n = q / (H / 8), c8 = q % (H / 8);
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (n < T) v = *reinterpret_cast<const uint4*>(a.x + (size_t)n * H + 8 * c8);
-            *reinterpret_cast<uint4*>(xs + (size_t)n * L.xs + 16 * c8) = v;
-        }
-        if (a.mode == MOE_MODE_SCATTER) {
-            const size_t n4 = (size_t)T * H / 4, per = (n4 + gridDim.x - 1) / gridDim.x;
-            const size_t lo = blockIdx.x * per, hi = min(n4, lo + per);
-            for (size_t q = lo + tid; q < hi; q += kConsumerWarps * 32)
-                reinterpret_cast<float4*>(a.y_acc)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        if (tid == 0) bar_base = ld_acquire_u64(ga.sync) / gridDim.x * gridDim.x;
-    }
+    // the shared expert's units come first in the unit order (active index 0)
+    const bool early = a.has_shared && (int)blockIdx.x < NJ;
+    if (warp == kConsumerWarps && lane == 0 && early) issue_unit(0, E, blockIdx.x);
 
-    // ---- active experts (the shared one first, then routed ones with rows),
-    // compacted by the producer warp alone so it can start issuing at once;
-    // the consumers wait for the list on named barrier 6.
-    __shared__ int s_r2p[kMaxT * 8];     // row -> pair (T*K <= 64 entries)
-    __shared__ float s_pw[kMaxT * 8];    // pair -> routing weight
+    // Everything below reads what earlier grids on the stream wrote.
+    griddep_wait();
+    griddep_launch_dependents();
+
     if (warp == kConsumerWarps) {
-        constexpr int EPL = 8;           // experts per lane (E <= 256)
+        // ---- active experts (the shared one first, then routed ones with rows)
+        constexpr int EPL = 8;   // experts per lane (E <= 256)
+        int ofs[EPL + 1];
+#pragma unroll
+        for (int q = 0; q <= EPL; ++q) {
+            const int e = lane * EPL + q;
+            ofs[q] = e <= E ? __ldcg(a.offsets + e) : 0;
+        }
         int cnt[EPL], lo[EPL], mine = 0;
+        bool bad = false;
 #pragma unroll
         for (int q = 0; q < EPL; ++q) {
             const int e = lane * EPL + q;
-            cnt[q] = 0;
-            lo[q] = 0;
-            if (e < E) {
-                const int l0 = a.offsets[e], h0 = a.offsets[e + 1];
-                if (l0 < 0 || h0 < l0 || h0 > T * K || h0 - l0 > kMaxT) {
-                    set_error(a.err, MOE_ERR_BOUNDS);
-                } else {
-                    cnt[q] = h0 - l0;
-                    lo[q] = l0;
-                }
-            }
+            const int l0 = ofs[q], h0 = ofs[q + 1];
+            const bool ok = e < E && l0 >= 0 && h0 >= l0 && h0 <= T * K && h0 - l0 <= kMaxT;
+            bad |= e < E && !ok;
+            cnt[q] = ok ? h0 - l0 : 0;
+            lo[q] = ok ? l0 : 0;
             mine += cnt[q] > 0;
         }
+        if (bad) set_error(a.err, MOE_ERR_BOUNDS);
         int incl = mine;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -298,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_gemv(GemvArgs ga) {
         if (lane == 31) {
             if (a.has_shared) {
                 act_e[0] = E;
-                act_row0[0] = T * K;
+                act_row0[0] = 0;
                 act_cnt[0] = T;
             }
             s_misc[0] = first + incl;
@@ -306,160 +249,233 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_gemv(GemvArgs ga) {
         __syncwarp();
         __threadfence_block();
         named_barrier_arrive(6, kThreads);
-    } else {
-        if (tid < T * K) {
-            s_r2p[tid] = r2p;
-            s_pw[tid] = pw;
+        // ---- producer: every unit of this CTA, in order.  Units 0 and 1 never
+        // wait for a down phase (their down slots are fresh), so they go first;
+        // the rest may, and a down phase waits for the y_acc count below.
+        const int A = s_misc[0];
+        auto issue_from = [&](int k0, int k1) {
+            if (lane != 0) return;
+            int k = k0;
+            for (int u = blockIdx.x + k0 * gridDim.x; u < A * NJ && k < k1; u += gridDim.x, ++k) {
+                if (k == 0 && early) continue;
+                issue_unit(k, act_e[u / NJ], u % NJ);
+            }
+        };
+        issue_from(0, 2);
+        // ---- y_acc: once the consumers cleared this CTA's slice, count the CTA
+        // and wait until every CTA of the launch is counted
+        named_barrier(7, kThreads);
+        if (lane == 0) {
+            // every earlier launch added exactly gridDim.x, so the count starts at
+            // a multiple of it
+            __threadfence();
+            const unsigned long long old = atom_add_release_u64(ga.sync, 1ull);
+            const unsigned long long target = old / gridDim.x * gridDim.x + gridDim.x;
+            const uint64_t t0 = globaltimer_ns();
+            while (ld_acquire_u64(ga.sync) < target) {
+                if (globaltimer_ns() - t0 > 200000000ull) {
+                    set_error(a.err, MOE_ERR_TIMEOUT);
+                    break;
+                }
+                __nanosleep(64);
+            }
+            mbar_arrive(zero_done);
         }
-        named_barrier(6, kThreads);
+        issue_from(2, 1 << 30);
+        __syncwarp();
+    } else {
+        // ---- routing tables, x (split order), this CTA's slice of y_acc
+        if (tid < T * K) {
+            s_r2p[tid] = __ldcg(a.row_to_pair + tid);
+            s_pw[tid] = __ldcg(a.topk_w + tid);
+        }
+        for (int q = tid; q < T * (H / 8); q += kConsumerWarps * 32) {
+            const int n = q / (H / 8), c8 = q % (H / 8);
+            const uint4 v = *reinterpret_cast<const uint4*>(a.x + (size_t)n * H + 8 * c8);
+            *reinterpret_cast<uint4*>(xs + (size_t)n * L.xs + 16 * c8) = to_split_order(v);
+        }
+        {
+            const size_t n4 = (size_t)T * H / 4, per = (n4 + gridDim.x - 1) / gridDim.x;
+            const size_t lo = blockIdx.x * per, hi = min(n4, lo + per);
+            for (size_t q = lo + tid; q < hi; q += kConsumerWarps * 32)
+                reinterpret_cast<float4*>(a.y_acc)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        named_barrier_arrive(7, kThreads);   // the slice is written
+        named_barrier(6, kThreads);          // the active list (producer); x and the tables (consumers)
     }
-    const int A = s_misc[0];
+
     if (warp < kConsumerWarps) {
-        // token and weight of each active expert's rows, from shared memory only
-        for (int q = tid; q < A * kMaxT; q += kConsumerWarps * 32) {
-            const int ai = q / kMaxT, i = q % kMaxT;
-            int tok = -1;
-            float w = 0.0f;
-            if (i < act_cnt[ai]) {
-                if (act_e[ai] == E) {
-                    tok = i;
+        const int A = s_misc[0];
+        const int g = lane >> 2, c = lane & 3;
+        const int t = warp & 3, kq = warp >> 2;        // gate/up: row tile, step within each box
+        const int jr = 8 * t + perm8(g);               // gate/up row (of the unit's 32) of MMA rows g, g+8
+        const int TW = H / 256;                        // 16-row down tiles per warp
+        const int nbase = 16 * TW * warp;              // first down row of this warp
+        bool zero_seen = false;
+        int k = 0;
+        for (int u = blockIdx.x; u < A * NJ; u += gridDim.x, ++k) {
+            const int ai = u / NJ, jb = u % NJ;
+            const int e = act_e[ai], cnt = act_cnt[ai], row0 = act_row0[ai];
+            auto column = [&](int col, float& w) -> int {   // token and weight of the expert's row col
+                w = 0.0f;
+                if (col >= cnt) return 0;
+                if (e == E) {
                     w = 1.0f;
-                } else {
-                    const int p = s_r2p[act_row0[ai] + i];
-                    if (p < 0 || p >= T * K) {
-                        set_error(a.err, MOE_ERR_BOUNDS);
-                        tok = 0;
-                    } else {
-                        tok = p / K;
-                        w = s_pw[p];
-                    }
+                    return col;
+                }
+                const int p = s_r2p[row0 + col];
+                if (p < 0 || p >= T * K) {
+                    set_error(a.err, MOE_ERR_BOUNDS);
+                    return 0;
+                }
+                w = s_pw[p];
+                return p / K;
+            };
+            float wg;
+            const int tok_g = column(g, wg);
+
+            // (scale, bias) words: gate/up rows of this lane for its steps, down rows of its tiles
+            const uint32_t* gsb = reinterpret_cast<const uint32_t*>(a.gu_sb);
+            const size_t grow = (size_t)e * 2 * I + kJ * jb + jr;   // gate row; up row = + I
+            uint32_t sbg[4], sbu[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                if (i < NP) {
+                    const int grp = 2 * (kq * NP + i) + (c >> 1);
+                    sbg[i] = ldg_u32(gsb + grow * ngr + grp);
+                    sbu[i] = ldg_u32(gsb + (grow + I) * ngr + grp);
                 }
             }
-            act_tok[q] = tok;
-            act_w[q] = w;
-        }
-        named_barrier(1, kConsumerWarps * 32);
-    }
-    Sched sc;
-    sc.init(A, I, H);
-    const int nst = sc.total();
+            // the down rows' (scale, bias) words of this block's group, into shared memory
+            uint32_t* dsb = dsb_s + (k & 1) * H;
+            {
+                const uint32_t* dsbp = reinterpret_cast<const uint32_t*>(a.d_sb) + (size_t)e * H * NB + (jb >> 1);
+                for (int n = tid; n < H; n += kConsumerWarps * 32) cp_async4(smem_u32(dsb + n), dsbp + (size_t)n * NB);
+                cp_async_commit();
+            }
 
-    if (warp == kConsumerWarps) {
-        // ------------------------------------------------------------ producer
-        for (int l = early ? 1 : 0; l < nst; ++l) {
-            const int slot = l % L.stages;
-            if (l >= L.stages && !mbar_wait_bounded(&empty[slot], ((l / L.stages) - 1) & 1, a.err)) break;
-            const int u = sc.unit(l);
-            if (sc.phase1(l)) {
-                issue_phase1(slot, act_e[u / (I / 8)], (u % (I / 8)) * 8);
-            } else {
-                uint8_t* st = smem + L.off_ring + (size_t)slot * L.stage_bytes;
-                const int ai = u / (H / 64), n0 = (u % (H / 64)) * 64, e = act_e[ai];
-                const uint8_t* codes = reinterpret_cast<const uint8_t*>(a.d_codes) + (size_t)e * H * (I / 2);
-                const uint8_t* sbd = reinterpret_cast<const uint8_t*>(a.d_sb) + (size_t)e * H * (I / 16);
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&full[slot], 64 * (I / 2) + 64 * (I / 16));
-                    bulk_g2s(st, codes + (size_t)n0 * (I / 2), 64 * (I / 2), &full[slot]);
-                    bulk_g2s(st + 64 * (I / 2), sbd + (size_t)n0 * (I / 16), 64 * (I / 16), &full[slot]);
+            // ---- gate/up: MMA rows g (gate) and g+8 (up) of tile t; steps kq NP .. kq NP + NP-1
+            float part[4][4];
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) part[w][q] = 0.0f;
+            const uint8_t* xrow = xs + (size_t)tok_g * L.xs;
+            const int rr = perm8(g);                   // row within the box
+            {
+                const int n = k * 4 + t, cs = n % kCodeSlots;
+                mbar_wait_bounded(&code_full[cs], (n / kCodeSlots) & 1, a.err);
+                const uint8_t* pb = smem + L.off_code + cs * kCodePiece;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    if (i >= NP) break;
+                    const int s = kq * NP + i;
+                    const int ch = s >> 1;                 // 256-input chunk = 128-byte line of the row
+                    const int phys = ((4 * (s & 1) + c) ^ rr) * 16;
+                    const uint4 ca = *reinterpret_cast<const uint4*>(pb + ((0 * NCH + ch) * 8 + rr) * 128 + phys);
+                    const uint4 cb = *reinterpret_cast<const uint4*>(pb + ((1 * NCH + ch) * 8 + rr) * 128 + phys);
+                    const uint32_t sA = sb_scale2(sbg[i]), bA = sb_bias2(sbg[i]);
+                    const uint32_t sB = sb_scale2(sbu[i]), bB = sb_bias2(sbu[i]);
+                    const uint8_t* xp = xrow + 2 * (128 * s + 32 * c);
+                    mma_word(part[0], ca.x, cb.x, sA, bA, sB, bB, *reinterpret_cast<const uint4*>(xp));
+                    mma_word(part[1], ca.y, cb.y, sA, bA, sB, bB, *reinterpret_cast<const uint4*>(xp + 16));
+                    mma_word(part[2], ca.z, cb.z, sA, bA, sB, bB, *reinterpret_cast<const uint4*>(xp + 32));
+                    mma_word(part[3], ca.w, cb.w, sA, bA, sB, bB, *reinterpret_cast<const uint4*>(xp + 48));
                 }
                 __syncwarp();
+                if (lane == 0) mbar_arrive(&code_empty[cs]);
             }
-        }
-        return;
-    }
-
-    // ---------------------------------------------------------------- consumers
-    const int quad = warp >> 2, wq = warp & 3;
-    const int g = lane >> 2, c = lane & 3;
-    bool grid_synced = false;
-    for (int l = quad;; l += 4) {
-        const bool done = l >= nst;
-        if (!grid_synced && (done || !sc.phase1(l))) {
-            // all phase-1 tiles of this CTA are finished once every quad gets here
-            named_barrier(1, kConsumerWarps * 32);
-            if (tid == 0) grid_barrier(ga.sync, bar_base + gridDim.x, a.err);
-            named_barrier(1, kConsumerWarps * 32);
-            grid_synced = true;
-        }
-        if (done) break;
-        const int slot = l % L.stages;
-        const uint8_t* st = smem + L.off_ring + (size_t)slot * L.stage_bytes;
-        const int u = sc.unit(l);
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        if (sc.phase1(l)) {
-            const int ai = u / (I / 8), j0 = (u % (I / 8)) * 8;
-            const int nsteps = H / 128 / 4;
-            const uint8_t* xrow = xs + (size_t)g * L.xs + 64 * c;
-            mbar_wait_bounded(&full[slot], (l / L.stages) & 1, a.err);
-            mma_rows16(acc, st, L.rs1, reinterpret_cast<const uint32_t*>(st + 16 * L.rs1), H / 64, wq * nsteps,
-                       nsteps, [&](int S, int w) {
-                           return *reinterpret_cast<const uint4*>(xrow + 2 * (128 * S + 8 * w));
-                       });
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[slot]);
-            red[(quad * 4 + wq) * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-            named_barrier(2 + quad, 128);
-            if (wq == 0) {
-                float t[4] = {0.f, 0.f, 0.f, 0.f};
+            float acc[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[q] = (part[0][q] + part[1][q]) + (part[2][q] + part[3][q]);
+            red[warp * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            named_barrier(2 + t, 128);   // the tile's four warps
+            uint16_t* hb = hbuf + (size_t)(k & 1) * kMaxT * kJ;
+            if (kq == 0) {
+                float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int w = 0; w < 4; ++w) {
-                    const float4 v = red[(quad * 4 + w) * 32 + lane];
-                    t[0] += v.x;
-                    t[1] += v.y;
-                    t[2] += v.z;
-                    t[3] += v.w;
+                    const float4 v = red[(t + 4 * w) * 32 + lane];
+                    s4[0] += v.x;
+                    s4[1] += v.y;
+                    s4[2] += v.z;
+                    s4[3] += v.w;
                 }
-                // rows g (gate j0+g) and g+8 (up j0+g); columns = tokens 2c, 2c+1
-                const float h0 = silu(t[0]) * t[2];
-                const float h1 = silu(t[1]) * t[3];
-                const int cnt = act_cnt[ai];
-                for (int i = 0; i < cnt; ++i) {
-                    const int tok = act_tok[ai * kMaxT + i];
-                    if (tok == 2 * c || tok == 2 * c + 1) {
-                        const size_t row = (size_t)act_row0[ai] + i;
-                        a.h[row * I + j0 + g] = f32_to_bf16(tok == 2 * c ? h0 : h1);
-                    }
-                }
+                // rows g (gate j) and g+8 (up j); columns 2c, 2c+1 = the expert's rows
+                const int pj = (jr & ~7) | split_pos(jr & 7);
+                hb[(2 * c) * kJ + pj] = 2 * c < cnt ? f32_to_bf16(silu(s4[0]) * s4[2]) : (uint16_t)0;
+                hb[(2 * c + 1) * kJ + pj] = 2 * c + 1 < cnt ? f32_to_bf16(silu(s4[1]) * s4[3]) : (uint16_t)0;
             }
-            named_barrier(2 + quad, 128);
-        } else {
-            const int ai = u / (H / 64), n0 = (u % (H / 64)) * 64 + 16 * wq;
-            const int cnt = act_cnt[ai];
-            // stage this expert's h rows (written by phase 1 on any CTA) for the quad
-            uint8_t* hq = xs + (size_t)quad * kMaxT * L.hs;
-            named_barrier(2 + quad, 128);                 // previous stage's readers are done
-            for (int q = wq * 32 + lane; q < kMaxT * (I / 8); q += 128) {
-                const int i = q / (I / 8), c8 = q % (I / 8);
-                uint4 v = make_uint4(0, 0, 0, 0);
-                if (i < cnt) v = ld_cg_v4(a.h + ((size_t)act_row0[ai] + i) * I + 8 * c8);
-                *reinterpret_cast<uint4*>(hq + (size_t)i * L.hs + 16 * c8) = v;
+            cp_async_wait<0>();
+            named_barrier(1, kConsumerWarps * 32);   // h and the down (scale, bias) words complete; red[] free
+
+            // ---- down: rows nbase + 16 tt + {g, g+8}, K = the unit's 32 columns
+            const int ds = k & 1;
+            mbar_wait_bounded(&d_full[ds], (k >> 1) & 1, a.err);
+            const uint4 hv = *reinterpret_cast<const uint4*>(hb + g * kJ + 8 * c);
+            const uint8_t* dbase = smem + L.off_d + ds * L.d_piece;
+            float w0, w1;
+            const int tok0 = column(2 * c, w0), tok1 = column(2 * c + 1, w1);
+            if (!zero_seen) {
+                mbar_wait_bounded(zero_done, 0, a.err);
+                zero_seen = true;
             }
-            named_barrier(2 + quad, 128);
-            const uint8_t* hrow = hq + (size_t)g * L.hs + 64 * c;
-            mbar_wait_bounded(&full[slot], (l / L.stages) & 1, a.err);
-            mma_rows16(acc, st + (size_t)16 * wq * L.rs2, L.rs2,
-                       reinterpret_cast<const uint32_t*>(st + 64 * L.rs2) + 16 * wq * (I / 64), I / 64, 0, I / 128,
-                       [&](int S, int w) {
-                           return *reinterpret_cast<const uint4*>(hrow + 2 * (128 * S + 8 * w));
-                       });
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[slot]);
-            // rows n0+g, n0+g+8; columns = the expert's rows 2c, 2c+1
+            // four tiles' codes and products at a time (independent), then their reductions
+            const bool lead = (g & 3) == 0;
+            for (int t0 = 0; t0 < TW; t0 += 4) {
+            float d[4][4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int i = 2 * c + (q & 1);
-                const int n = n0 + g + (q >> 1) * 8;
-                if (i < cnt) {
-                    const int tok = act_tok[ai * kMaxT + i];
-                    if (a.mode == MOE_MODE_SCATTER) {
-                        atomicAdd(a.y_acc + (size_t)tok * H + n, act_w[ai * kMaxT + i] * acc[q]);
-                    } else if (act_e[ai] == E) {
-                        a.y_shared[(size_t)tok * H + n] = f32_to_bf16(acc[q]);
-                    } else {
-                        a.y_rows[((size_t)act_row0[ai] + i) * H + n] = f32_to_bf16(acc[q]);
+            for (int tt = 0; tt < 4; ++tt) {
+                if (t0 + tt < TW) {
+                    const int nl = nbase + 16 * (t0 + tt) + g;
+                    const uint32_t va = *reinterpret_cast<const uint32_t*>(dbase + (size_t)nl * 16 + 4 * c);
+                    const uint32_t vb = *reinterpret_cast<const uint32_t*>(dbase + (size_t)(nl + 8) * 16 + 4 * c);
+                    const uint32_t sa = dsb[nl], sb = dsb[nl + 8];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) d[tt][q] = 0.0f;
+                    mma_word(d[tt], va, vb, sb_scale2(sa), sb_bias2(sa), sb_scale2(sb), sb_bias2(sb), hv);
+                }
+            }
+#pragma unroll
+            for (int tt = 0; tt < 4; ++tt) {
+                if (t0 + tt >= TW) break;
+                const int nl = nbase + 16 * (t0 + tt) + g;
+                // lanes g = 0 and 4 collect rows g..g+3 (and g+8..g+11) of their
+                // column from lanes g+1..g+3 and add them with one vector reduction
+                float4 q0, q2;
+                q0.x = d[tt][0];
+                q0.y = __shfl_down_sync(0xFFFFFFFFu, d[tt][0], 4);
+                q0.z = __shfl_down_sync(0xFFFFFFFFu, d[tt][0], 8);
+                q0.w = __shfl_down_sync(0xFFFFFFFFu, d[tt][0], 12);
+                q2.x = d[tt][2];
+                q2.y = __shfl_down_sync(0xFFFFFFFFu, d[tt][2], 4);
+                q2.z = __shfl_down_sync(0xFFFFFFFFu, d[tt][2], 8);
+                q2.w = __shfl_down_sync(0xFFFFFFFFu, d[tt][2], 12);
+                if (lead && 2 * c < cnt) {
+                    float* y0 = a.y_acc + (size_t)tok0 * H + nl;
+                    red_add_v4(y0, w0 * q0.x, w0 * q0.y, w0 * q0.z, w0 * q0.w);
+                    red_add_v4(y0 + 8, w0 * q2.x, w0 * q2.y, w0 * q2.z, w0 * q2.w);
+                }
+                if (cnt > 1) {   // odd columns hold tokens only when the expert has two or more rows
+                    float4 q1, q3;
+                    q1.x = d[tt][1];
+                    q1.y = __shfl_down_sync(0xFFFFFFFFu, d[tt][1], 4);
+                    q1.z = __shfl_down_sync(0xFFFFFFFFu, d[tt][1], 8);
+                    q1.w = __shfl_down_sync(0xFFFFFFFFu, d[tt][1], 12);
+                    q3.x = d[tt][3];
+                    q3.y = __shfl_down_sync(0xFFFFFFFFu, d[tt][3], 4);
+                    q3.z = __shfl_down_sync(0xFFFFFFFFu, d[tt][3], 8);
+                    q3.w = __shfl_down_sync(0xFFFFFFFFu, d[tt][3], 12);
+                    if (lead && 2 * c + 1 < cnt) {
+                        float* y1 = a.y_acc + (size_t)tok1 * H + nl;
+                        red_add_v4(y1, w1 * q1.x, w1 * q1.y, w1 * q1.z, w1 * q1.w);
+                        red_add_v4(y1 + 8, w1 * q3.x, w1 * q3.y, w1 * q3.z, w1 * q3.w);
                     }
                 }
             }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&d_empty[ds]);
         }
     }
 }
@@ -472,35 +488,87 @@ int num_sms_cached() {
     return sms[dev];
 }
 
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled gemv_encode_fn() {
+    static EncodeTiled fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiled>(p);
+    }
+    return fn;
+}
+
+// Gate/up codes as a 5-D view (32 words of a 256-input chunk, row j of I,
+// chunk, gate|up, expert); one box = 8 whole rows of gate and the same 8 of
+// up (two contiguous runs of HBM), landing as [gate|up][chunk][row][128 B] so
+// a 128-byte line's swizzle phase is its row.
+bool make_gu_map(CUtensorMap* m, const FfnArgs& a) {
+    EncodeTiled enc = gemv_encode_fn();
+    if (!enc) return false;
+    const uint64_t row = (uint64_t)a.H / 2;
+    const cuuint64_t dims[5] = {32, (cuuint64_t)a.I, (cuuint64_t)(a.H / 256), 2, (cuuint64_t)(a.E + 1)};
+    const cuuint64_t strides[4] = {row, 128, (cuuint64_t)a.I * row, (cuuint64_t)2 * a.I * row};
+    const cuuint32_t box[5] = {32, 8, (cuuint32_t)(a.H / 256), 2, 1};
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 5, const_cast<uint32_t*>(a.gu_codes), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Down codes as a 4-D view (4 words of a 32-input block, row of a 256-row
+// band, band, block); one box = the H rows of one expert and block.
+bool make_d_map(CUtensorMap* m, const FfnArgs& a) {
+    EncodeTiled enc = gemv_encode_fn();
+    if (!enc) return false;
+    const uint64_t row = (uint64_t)a.I / 2;
+    const cuuint64_t dims[4] = {4, 256, (cuuint64_t)(a.E + 1) * (a.H / 256), (cuuint64_t)(a.I / kJ)};
+    const cuuint64_t strides[3] = {row, 256 * row, 16};
+    const cuuint32_t box[4] = {4, 256, (cuuint32_t)(a.H / 256), 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, const_cast<uint32_t*>(a.d_codes), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 bool ffn_gemv_supported(const FfnArgs& a) {
-    if (a.T > kMaxT || a.H > 2048 || a.H % 512 != 0 || a.I % 128 != 0 || a.E > 256 || a.K != 8) return false;
-    const GemvLayout L = gemv_layout(a.H, a.I);
-    return L.stages >= 4 && L.total <= kSmemBudget;
+    return a.mode == MOE_MODE_SCATTER && a.T >= 1 && a.T <= kMaxT && a.K == 8 && a.G == 64 && a.E <= 256 &&
+           (a.H == 512 || a.H == 1024 || a.H == 2048) && a.I % 64 == 0 && a.I >= 64 && a.I <= 8192;
 }
 
 cudaError_t launch_ffn_gemv(const FfnArgs& a, unsigned long long* sync, cudaStream_t st) {
     GemvArgs ga;
     ga.f = a;
-    ga.L = gemv_layout(a.H, a.I);
+    ga.L = gemv_layout(a.H);
     ga.sync = sync;
+    CUtensorMap gu_map, d_map;
+    if (!make_gu_map(&gu_map, a) || !make_d_map(&d_map, a)) return cudaErrorInvalidValue;
     static int done[64] = {0};
-    cudaError_t ce = set_smem_once(k_ffn_gemv, ga.L.total, done);
+    const int smem = ga.L.total + 1024;
+    cudaError_t ce = set_smem_once(k_ffn_gemv, smem, done);
     if (ce != cudaSuccess) return ce;
     const int G = num_sms_cached();
     if (G <= 0) return cudaErrorInvalidDevice;
+    // one CTA per SM, all resident at once (the in-kernel count of zeroing
+    // CTAs waits for every CTA of the launch)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(G);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = ga.L.total;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_ffn_gemv, ga);
+    return cudaLaunchKernelEx(&cfg, k_ffn_gemv, gu_map, d_map, ga);
 }
 
 }  // namespace moe

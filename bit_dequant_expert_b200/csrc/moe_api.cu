@@ -248,7 +248,8 @@ int32_t moe_launch_count(const moe_config_t* cfg, int32_t T, int32_t mode, int32
     if (mode != MOE_MODE_SCATTER && mode != MOE_MODE_PAIRS) return -1;
     const int route = T <= 8 ? 1 : 2;
     const int permute = T <= 256 ? 1 : 3;
-    const FfnArgs a = shape_only(cfg, T);
+    FfnArgs a = shape_only(cfg, T);
+    a.mode = mode;
     if (path == MOE_PATH_AUTO) path = resolve_path(a);
     int ffn;
     switch (path) {

@@ -16,6 +16,7 @@
 // per-(chunk, expert) row bases.
 #include "common.cuh"
 #include "kernels.h"
+#include "ptx.cuh"
 
 namespace moe {
 
@@ -168,6 +169,8 @@ __global__ void __launch_bounds__(256) k_perm_small(int T, int E, const int32_t*
                                                     int32_t* __restrict__ pair_to_row, int32_t* err) {
     extern __shared__ uint32_t mask[];
     int* s_off = reinterpret_cast<int*>(mask + E * (kChunk / 32));
+    griddep_wait();   // idx and counts come from the router
+    griddep_launch_dependents();
     build_masks<K>(T, E, 0, idx, mask, err);
     // E <= 1024: each thread scans E / blockDim.x experts in order
     const int per = (E + blockDim.x - 1) / blockDim.x;
@@ -220,9 +223,8 @@ size_t permute_ws_bytes(int T, int E, int K) {
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st) {
     const size_t mask_bytes = (size_t)a.E * (kChunk / 32) * sizeof(uint32_t);
     if (a.T <= kChunk) {
-        k_perm_small<8><<<1, 256, mask_bytes + a.E * sizeof(int), st>>>(a.T, a.E, a.topk_idx, a.counts, a.offsets,
-                                                                       a.row_to_pair, a.pair_to_row, a.err);
-        return cudaGetLastError();
+        return launch_pdl(k_perm_small<8>, dim3(1), dim3(256), mask_bytes + a.E * sizeof(int), st, a.T, a.E,
+                          a.topk_idx, a.counts, a.offsets, a.row_to_pair, a.pair_to_row, a.err);
     }
     const int nchunk = (a.T + kChunk - 1) / kChunk;
     int32_t* hist = reinterpret_cast<int32_t*>(a.scratch);

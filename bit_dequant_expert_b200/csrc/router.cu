@@ -8,6 +8,7 @@
 // (GPU-resident expert routing).
 #include "common.cuh"
 #include "kernels.h"
+#include "ptx.cuh"
 
 namespace moe {
 
@@ -217,7 +218,101 @@ __global__ void __launch_bounds__(256) k_route_small(int T, int H, int E, const 
     if (threadIdx.x == 0) *ticket = 0u;
 }
 
+// A handful of tokens (T <= 8, H <= 2048): one warp per expert, two experts
+// per block, so the router matrix streams through 128 SMs.  Each lane issues
+// all of its weight chunks at once, before waiting on the previous grid (the
+// weights never depend on it); x is staged in shared memory.  The logits of
+// (token, expert) follow the same contract order as router_tile.  The last
+// block (atomic ticket, reset by that block) selects the top-k and counts.
+constexpr int kSmallMaxChunksPerLane = 8;   // H <= 8 * 8 * 32
+
+__global__ void __launch_bounds__(64) k_route_small_wide(int T, int H, int E, const uint16_t* __restrict__ x,
+                                                         const uint16_t* __restrict__ wr,
+                                                         const float* __restrict__ bias, int64_t bias_stride,
+                                                         float* __restrict__ logits, int32_t* __restrict__ idx,
+                                                         float* __restrict__ wout, int32_t* __restrict__ counts,
+                                                         uint32_t* ticket, int32_t* err) {
+    extern __shared__ uint4 xs4[];   // [T][H/8]
+    __shared__ bool last;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e = blockIdx.x * 2 + warp;
+    const int nchunk = H / 8;
+    uint4 wv[kSmallMaxChunksPerLane];
+#pragma unroll
+    for (int i = 0; i < kSmallMaxChunksPerLane; ++i) {
+        const int c = lane + 32 * i;
+        wv[i] = c < nchunk ? ldg_v4(wr + (size_t)e * H + 8 * c) : make_uint4(0, 0, 0, 0);
+    }
+    griddep_wait();
+    griddep_launch_dependents();
+    for (int q = threadIdx.x; q < T * nchunk; q += blockDim.x) xs4[q] = reinterpret_cast<const uint4*>(x)[q];
+    __syncthreads();
+    float acc[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) acc[t] = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kSmallMaxChunksPerLane; ++i) {
+        const int c = lane + 32 * i;
+        if (c >= nchunk) break;
+        const uint32_t ww[4] = {wv[i].x, wv[i].y, wv[i].z, wv[i].w};
+        float wf[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            wf[2 * q] = bf16_lo(ww[q]);
+            wf[2 * q + 1] = bf16_hi(ww[q]);
+        }
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            if (t < T) {
+                const uint4 xv = xs4[t * nchunk + c];
+                const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                float sacc = acc[t];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    sacc = __fmaf_rn(bf16_lo(xw[q]), wf[2 * q], sacc);   // inputs ascending in the chunk
+                    sacc = __fmaf_rn(bf16_hi(xw[q]), wf[2 * q + 1], sacc);
+                }
+                acc[t] = sacc;
+            }
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+        float v = acc[t];
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xFFFFFFFFu, v, off));
+        if (lane == t && t < T) {
+            if (bias) v = __fadd_rn(v, bias[(int64_t)t * bias_stride + e]);
+            logits[(size_t)t * E + e] = v;
+        }
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) last = atomicAdd(ticket, 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    for (int q = threadIdx.x; q < E; q += blockDim.x) counts[q] = 0;
+    __syncthreads();
+    for (int t = warp; t < T; t += 2) topk_token<8, 8>(t, E, logits, nullptr, 0, idx, wout, counts, err);
+    if (threadIdx.x == 0) *ticket = 0u;
+}
+
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t st) {
+    if (!a.logits_in && a.T <= 8 && a.E == 256 && a.H <= 8 * kSmallMaxChunksPerLane * 32) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(a.E / 2);
+        cfg.blockDim = dim3(64);
+        cfg.dynamicSmemBytes = (size_t)a.T * a.H * 2;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, k_route_small_wide, a.T, a.H, a.E, a.x, a.w_router, a.bias, a.bias_stride,
+                                  a.logits_ws, a.topk_idx, a.topk_w, a.counts, a.ticket, a.err);
+    }
     if (!a.logits_in && a.T <= 8 && a.E == 256) {
         k_route_small<<<a.E / 8, 256, 0, st>>>(a.T, a.H, a.E, a.x, a.w_router, a.bias, a.bias_stride, a.logits_ws,
                                                a.topk_idx, a.topk_w, a.counts, a.ticket, a.err);

@@ -186,42 +186,63 @@ def test_permute_bitexact_random(T):
 # ------------------------------------------------------------ decode (GEMV) path
 
 
-@pytest.mark.parametrize("mode", [SCATTER, PAIRS])
 @pytest.mark.parametrize("T", [1, 2, 3, 5, 8])
-def test_gemv_small_shapes(T, mode):
+def test_gemv_small_shapes(T):
     lay = layer_of(0, T=T)
-    out, _ = run_layer(lay, mode, GEMV)
+    out, _ = run_layer(lay, SCATTER, GEMV)
     assert out["err"] == 0
     check_routing(out, lay)
     check_output(out, lay, np.arange(T))
 
 
-@pytest.mark.parametrize("mode", [SCATTER, PAIRS])
-def test_gemv_decode_layers(mode):
+def test_gemv_decode_layers():
     spec = gen.config(1)
     for layer in (0, 39):
         lay = gen.make_layer(spec, layer)
-        out, _ = run_layer(lay, mode, GEMV)
+        out, _ = run_layer(lay, SCATTER, GEMV)
         assert out["err"] == 0
         check_routing(out, lay)
         check_output(out, lay, [0])
 
 
+@pytest.mark.parametrize("T", [1, 6])
+def test_gemv_hidden_1024(T):
+    """H = 1024, I = 256: two code boxes per unit, two down tiles per warp,
+    four intermediate blocks per expert."""
+    spec = gen.LayerSpec(T=T, H=1024, I=256, seed=11)
+    lay = gen.make_layer(spec, 0)
+    out, _ = run_layer(lay, SCATTER, GEMV)
+    assert out["err"] == 0
+    check_routing(out, lay)
+    check_output(out, lay, np.arange(T))
+
+
+def test_gemv_rejects_pairs_mode():
+    """The decode kernel accumulates split-K partial sums, so it only writes
+    y_acc; asked for bf16 rows it declines before launching."""
+    import bit_dequant_expert_b200 as m
+    lay = layer_of(0, T=2)
+    with pytest.raises(m.MoeError) as ex:
+        run_layer(lay, PAIRS, GEMV)
+    assert ex.value.status == m.MOE_ERR_UNSUPPORTED
+
+
 @pytest.mark.parametrize("T", [4, 8])
 def test_gemv_matches_simt_and_repeats(T):
     """The decode kernel agrees with the CUDA-core path, and repeated calls
-    (which reuse the grid-barrier words) give identical results."""
+    (which reuse the arrival counter) stay correct: the fp32 accumulation
+    order may differ between calls, nothing else."""
     import torch
     from bit_dequant_expert_b200.layer import MoELayer, to_device
     lay = layer_of(3, T=T)
-    Lg = MoELayer(lay, max_tokens=T, path=GEMV, mode=PAIRS)
+    Lg = MoELayer(lay, max_tokens=T, path=GEMV, mode=SCATTER)
     Ls = MoELayer(lay, max_tokens=T, path=SIMT, mode=PAIRS)
     x = to_device(lay["x"], "cuda")
     ys = Ls.forward(x).float().cpu().numpy()
     first = Lg.forward(x).float().cpu().numpy().copy()
     for _ in range(5):
         again = Lg.forward(x).float().cpu().numpy()
-        assert np.array_equal(again, first)
+        assert np.max(row_rel_err(again.astype(np.float64), first.astype(np.float64))) < 1e-2
     torch.cuda.synchronize()
     import bit_dequant_expert_b200 as m
     assert m.moe_get_device_error(Lg.ws) == 0
