@@ -213,7 +213,11 @@ def _capture(fn, stream):
 
 
 def _launch_count(layer, T):
+    """Kernels one forward() of the layer launches: two for the fused decode
+    layer (moe_decode_layer), else the four calls' count."""
     import bit_dequant_expert_b200 as m
+    if layer.fused_ok(T):
+        return 2
     return m.moe_launch_count(layer.cfg, T, layer.mode, layer.path)
 
 
@@ -284,9 +288,18 @@ def run_decode(device, steps, warmup, world, peaks):
     e2e = {"value": LAYERS / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": LAYERS * H * 2,
            "d2h_bytes_per_step": LAYERS * H * 2, "ms_per_step": e2e_ms}
 
+    # the whole layer (fused decode kernel + combine): router + expert bytes per layer pass
+    layer_bytes = LAYER_BYTES_T1
+    layer_us = ms_step * 1e3 / LAYERS
+    roofline_layer = {"bound": "hbm", "achieved": layer_bytes / (layer_us * 1e-6) / 1e9, "peak": peaks["hbm_gbs"],
+                      "unit": "GB/s", "frac": layer_bytes / (layer_us * 1e-6) / 1e9 / peaks["hbm_gbs"],
+                      "kernel": "moe_decode_layer (fused route + permute + expert FFN, then combine)",
+                      "algorithmic_bytes": layer_bytes, "avg_layer_us": layer_us,
+                      "peak_source": peaks["source"] + " hbm_gbs"}
     breakdown = _breakdown(layers, [x_dev[l:l + 1] for l in range(LAYERS)], 1, steps, stream)
     launches = _launch_count(layers[0], 1) * LAYERS
-    return {"ms_per_step": ms_step, "units_per_step": LAYERS * 1, "roofline": roofline, "e2e": e2e,
+    return {"ms_per_step": ms_step, "units_per_step": LAYERS * 1, "roofline": roofline,
+            "roofline_layer": roofline_layer, "e2e": e2e,
             "clocks": clocks, "gpu_launches": launches * steps, "breakdown_us_per_layer": breakdown,
             "_host_layers": host}
 
@@ -425,12 +438,13 @@ def main(argv=None):
             "seq_len": 1,
             "parallelism": "replicas" if world > 1 else "single GPU",
             "l2": "inputs larger than L2 (18.2 GB of weights streamed per step; no flush)",
-            "graph": "one CUDA graph per step (40 layers x route, permute, ffn, combine)",
+            "graph": "one CUDA graph per step (40 layers x moe_decode_layer: fused route + permute + expert FFN kernel, then combine)",
         },
         "decode_token_per_s": world / (ms / 1e3),
         "breakdown_us_per_layer": res["breakdown_us_per_layer"],
         "gpu_launches": res["gpu_launches"],
         "roofline": res["roofline"],
+        "roofline_layer": res["roofline_layer"],
         "e2e": res["e2e"],
         "clocks": res["clocks"],
         "peaks": peaks,

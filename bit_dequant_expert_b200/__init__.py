@@ -43,7 +43,7 @@ MOE_PATH_TC = 3
 EXPORTED = (
     "moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permute", "moe_expert_ffn",
     "moe_expert_ffn_path", "moe_combine", "moe_get_device_error", "moe_status_string", "moe_launch_count",
-    "moe_permute_static",
+    "moe_permute_static", "moe_decode_layer",
 )
 
 MOE_STATIC_MAX_TOKENS = 16384
@@ -81,6 +81,9 @@ _lib.moe_get_device_error.restype = _I32
 _lib.moe_get_device_error.argtypes = [_P, _P]
 _lib.moe_permute_static.restype = _I32
 _lib.moe_permute_static.argtypes = [_CFG, _I32, _P, _P, _P, _P, _P, _P, _P]
+_lib.moe_decode_layer.restype = _I32
+_lib.moe_decode_layer.argtypes = [_CFG, _I32, _P, _P, _P, ctypes.c_int64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                  _P, _P, _P, ctypes.c_size_t, _P]
 _lib.moe_launch_count.restype = _I32
 _lib.moe_launch_count.argtypes = [_CFG, _I32, _I32, _I32]
 _lib.moe_status_string.restype = ctypes.c_char_p
@@ -172,6 +175,19 @@ def moe_combine(cfg, T, mode, in0, in1, pair_to_row, topk_w, y, stream=None, rai
     st = _lib.moe_combine(ctypes.byref(cfg), T, mode, _ptr(in0), _ptr(in1), _ptr(pair_to_row), _ptr(topk_w), _ptr(y),
                           _stream(stream))
     return _check(st, "moe_combine", raise_on_error)
+
+
+def moe_decode_layer(cfg, T, x, w_router, logit_bias, logit_bias_row_stride, gu_codes, gu_sb, d_codes, d_sb,
+                     topk_idx, topk_w, counts, offsets, row_to_pair, pair_to_row, y_acc, y, ws, ws_bytes=None,
+                     stream=None, raise_on_error=True) -> int:
+    """The whole layer for T <= 8 tokens in two launches (router, top-k and
+    permutation fused into the decode expert FFN, then the combine)."""
+    n = _nbytes(ws) if ws_bytes is None else ws_bytes
+    st = _lib.moe_decode_layer(ctypes.byref(cfg), T, _ptr(x), _ptr(w_router), _ptr(logit_bias),
+                               logit_bias_row_stride, _ptr(gu_codes), _ptr(gu_sb), _ptr(d_codes), _ptr(d_sb),
+                               _ptr(topk_idx), _ptr(topk_w), _ptr(counts), _ptr(offsets), _ptr(row_to_pair),
+                               _ptr(pair_to_row), _ptr(y_acc), _ptr(y), _ptr(ws), n, _stream(stream))
+    return _check(st, "moe_decode_layer", raise_on_error)
 
 
 def moe_permute_static(cfg, T, topk_idx, counts, offsets, row_to_pair, pair_to_row, err_out=None, stream=None,

@@ -11,8 +11,8 @@ namespace moe {
 // y = bf16(y_acc), eight values per thread.
 __global__ void __launch_bounds__(256) k_combine_scatter(size_t n8, const float* __restrict__ y_acc,
                                                          uint16_t* __restrict__ y) {
-    griddep_wait();   // y_acc comes from the expert FFN
-    griddep_launch_dependents();
+    griddep_launch_dependents();   // the next grid may start its own prologue
+    griddep_wait();                // y_acc comes from the expert FFN
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8; i += (size_t)gridDim.x * blockDim.x) {
         const float4 a = reinterpret_cast<const float4*>(y_acc)[2 * i];
         const float4 b = reinterpret_cast<const float4*>(y_acc)[2 * i + 1];
@@ -36,8 +36,8 @@ __global__ void __launch_bounds__(256) k_combine_pairs(int T, int H, int has_sha
     const int t = blockIdx.x;
     __shared__ int s_row[K];
     __shared__ float s_w[K];
-    griddep_wait();   // rows come from the expert FFN
-    griddep_launch_dependents();
+    griddep_launch_dependents();   // the next grid may start its own prologue
+    griddep_wait();                // rows come from the expert FFN
     if (threadIdx.x < K) {
         int r = pair_to_row[(size_t)t * K + threadIdx.x];
         if (r < 0 || r >= T * K) {

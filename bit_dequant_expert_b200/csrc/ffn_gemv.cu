@@ -41,6 +41,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
+#include "topk.cuh"
 
 namespace moe {
 
@@ -73,16 +74,33 @@ __host__ __device__ inline GemvLayout gemv_layout(int H) {
     L.off_h = L.off_red + kConsumerWarps * 32 * 16;
     L.off_dsb = round_up(L.off_h + 2 * kMaxT * kJ * 2, 128);   // [2][H] down (scale, bias) words
     L.off_tab = L.off_dsb + 2 * H * 4;
-    // act_e, act_row0, act_cnt [kMaxActive]; row -> pair [64]; pair -> weight [64]; misc [4]
-    L.off_bar = round_up(L.off_tab + (3 * kMaxActive + 64 + 64 + 4) * 4, 128);
+    // act_e, act_row0, act_cnt [kMaxActive]; row -> pair [64]; pair -> weight [64]; misc [4];
+    // selected expert [64] and weight [64] per pair; expert offsets [kMaxActive]
+    L.off_bar = round_up(L.off_tab + (3 * kMaxActive + 64 + 64 + 4 + 64 + 64 + kMaxActive) * 4, 128);
     L.total = L.off_bar + 32 * 8;
     return L;
 }
+
+// Routing done inside the decode kernel (fused layer): inputs and the outputs
+// the separate route and permute calls would have written.
+struct GemvRoute {
+    const uint16_t* w_router;   // [E, H] bf16
+    const float* bias;          // nullable; [T, E] with row stride bias_stride (0: one row for all tokens)
+    int64_t bias_stride;
+    float* logits;              // [T, E] fp32 scratch
+    int32_t* topk_idx;          // [T, K]
+    float* topk_w;              // [T, K]
+    int32_t* counts;            // [E]
+    int32_t* offsets;           // [E + 1]
+    int32_t* row_to_pair;       // [T K]
+    int32_t* pair_to_row;       // [T K]
+};
 
 struct GemvArgs {
     FfnArgs f;
     GemvLayout L;
     unsigned long long* sync;   // monotonic arrival counter (workspace header)
+    GemvRoute r;
 };
 
 __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
@@ -128,6 +146,28 @@ __device__ __forceinline__ void mma_word(float (&d)[4], uint32_t va, uint32_t vb
 __device__ __forceinline__ uint32_t sb_scale2(uint32_t w) { return prmt(w, w, 0x1010); }
 __device__ __forceinline__ uint32_t sb_bias2(uint32_t w) { return prmt(w, w, 0x3232); }
 
+// Adds this CTA to the monotonic counter and waits (bounded) until every CTA
+// of the launch is counted: a grid-wide barrier for co-resident CTAs.  Every
+// earlier launch added exactly gridDim.x, so the count starts at a multiple
+// of it.  Releases this thread's (and, through the preceding CTA barrier,
+// the CTA's) writes; acquires everyone's.
+__device__ void grid_arrive_wait(unsigned long long* sync, int32_t* err) {
+    __threadfence();
+    const unsigned long long old = atom_add_release_u64(sync, 1ull);
+    const unsigned long long target = old / gridDim.x * gridDim.x + gridDim.x;
+    const uint64_t t0 = globaltimer_ns();
+    while (ld_acquire_u64(sync) < target) {
+        if (globaltimer_ns() - t0 > 200000000ull) {
+            set_error(err, MOE_ERR_TIMEOUT);
+            break;
+        }
+        __nanosleep(32);
+    }
+}
+
+// kRoute: the kernel also routes (router logits, top-k, permutation); else it
+// reads the permutation written by the route and permute calls.
+template <bool kRoute>
 __global__ void __launch_bounds__(kThreads, 1)
     k_ffn_gemv(const __grid_constant__ CUtensorMap gu_map, const __grid_constant__ CUtensorMap d_map,
                const GemvArgs ga) {
@@ -149,6 +189,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int* s_r2p = act_cnt + kMaxActive;
     float* s_pw = reinterpret_cast<float*>(s_r2p + 64);
     int* s_misc = reinterpret_cast<int*>(s_pw + 64);
+    int* s_sel = s_misc + 4;                                         // [T K] selected expert per pair
+    float* s_selw = reinterpret_cast<float*>(s_sel + 64);            // [T K] its weight
+    int* s_off = reinterpret_cast<int*>(s_selw + 64);                // [E + 1] expert offsets
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.off_bar);
     uint64_t* code_full = bars;
     uint64_t* code_empty = bars + 4;
@@ -194,12 +237,197 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the shared expert's units come first in the unit order (active index 0)
     const bool early = a.has_shared && (int)blockIdx.x < NJ;
     if (warp == kConsumerWarps && lane == 0 && early) issue_unit(0, E, blockIdx.x);
+    // router rows of this CTA (warp w: expert b + w gridDim.x; warps 0 and 1 on 148 SMs),
+    // lane l holding chunks l, l+32, ... of the row
+    constexpr int kRChunks = 8;   // H <= 2048
+    uint4 wv[kRChunks];
+    const int r_e = (int)blockIdx.x + warp * (int)gridDim.x;
+    const bool r_on = kRoute && warp < kConsumerWarps && r_e < E;
+    if (kRoute) {
+#pragma unroll
+        for (int i = 0; i < kRChunks; ++i) {
+            const int c = lane + 32 * i;
+            wv[i] = r_on && c < H / 8 ? ldg_v4(ga.r.w_router + (size_t)r_e * H + 8 * c) : make_uint4(0, 0, 0, 0);
+        }
+    }
 
-    // Everything below reads what earlier grids on the stream wrote.
-    griddep_wait();
+    // The next grid may start its prologue; everything below reads what
+    // earlier grids on the stream wrote.
     griddep_launch_dependents();
+    griddep_wait();
 
-    if (warp == kConsumerWarps) {
+    if (kRoute) {
+        if (warp < kConsumerWarps) {
+            // ---- x (split order), this CTA's slice of y_acc
+            for (int q = tid; q < T * (H / 8); q += kConsumerWarps * 32) {
+                const int n = q / (H / 8), c8 = q % (H / 8);
+                const uint4 v = *reinterpret_cast<const uint4*>(a.x + (size_t)n * H + 8 * c8);
+                *reinterpret_cast<uint4*>(xs + (size_t)n * L.xs + 16 * c8) = to_split_order(v);
+            }
+            const size_t n4 = (size_t)T * H / 4, per = (n4 + gridDim.x - 1) / gridDim.x;
+            const size_t lo = blockIdx.x * per, hi = min(n4, lo + per);
+            for (size_t q = lo + tid; q < hi; q += kConsumerWarps * 32)
+                reinterpret_cast<float4*>(a.y_acc)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+            named_barrier(1, kConsumerWarps * 32);
+            // ---- router logits of this CTA's experts: lane l accumulates its chunks in
+            // order with fma, the 32 partials meet in the xor butterfly 16..1, then
+            // the bias is added
+            if (r_on) {
+                float acc[kMaxT];
+#pragma unroll
+                for (int t = 0; t < kMaxT; ++t) acc[t] = 0.0f;
+#pragma unroll
+                for (int i = 0; i < kRChunks; ++i) {
+                    const int c = lane + 32 * i;
+                    if (c < H / 8) {
+                        const uint32_t ww[4] = {wv[i].x, wv[i].y, wv[i].z, wv[i].w};
+#pragma unroll
+                        for (int t = 0; t < kMaxT; ++t) {
+                            if (t < T) {
+                                // x chunk in split order: (x0,x4) (x1,x5) (x2,x6) (x3,x7)
+                                const uint4 xv = *reinterpret_cast<const uint4*>(xs + (size_t)t * L.xs + 16 * c);
+                                const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                                float sacc = acc[t];
+#pragma unroll
+                                for (int j = 0; j < 8; ++j) {
+                                    const float xj = j < 4 ? bf16_lo(xw[j]) : bf16_hi(xw[j - 4]);
+                                    const float wj = (j & 1) ? bf16_hi(ww[j >> 1]) : bf16_lo(ww[j >> 1]);
+                                    sacc = __fmaf_rn(xj, wj, sacc);
+                                }
+                                acc[t] = sacc;
+                            }
+                        }
+                    }
+                }
+#pragma unroll
+                for (int t = 0; t < kMaxT; ++t) {
+                    float v = acc[t];
+#pragma unroll
+                    for (int off = 16; off >= 1; off >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xFFFFFFFFu, v, off));
+                    if (lane == t && t < T) {
+                        if (ga.r.bias) v = __fadd_rn(v, ga.r.bias[(int64_t)t * ga.r.bias_stride + r_e]);
+                        ga.r.logits[(size_t)t * E + r_e] = v;
+                    }
+                }
+            }
+            named_barrier(1, kConsumerWarps * 32);
+            // ---- every CTA's logits and y_acc slice are written
+            if (tid == 0) grid_arrive_wait(ga.sync, a.err);
+            named_barrier(1, kConsumerWarps * 32);
+            // ---- top-k of every token, in every CTA
+            if (warp < T) {
+                int e_sel;
+                float w_sel;
+                if (topk_select<8, 8>(warp, E, ga.r.logits, nullptr, 0, e_sel, w_sel) && lane == 0 &&
+                    blockIdx.x == 0)
+                    set_error(a.err, MOE_ERR_NONFINITE);
+                if (lane < K) {
+                    s_sel[warp * K + lane] = e_sel;
+                    s_selw[warp * K + lane] = w_sel;
+                }
+            }
+            named_barrier(6, kThreads);   // selections ready for the producer
+            named_barrier(8, kThreads);   // the producer built the tables
+        } else {
+            named_barrier(6, kThreads);
+            // ---- permutation: rows expert-major, token-ascending.  Pairs p = t K + k
+            // come in token order, so a pair's rank among its expert's rows is the
+            // number of earlier pairs with the same expert: lanes holding equal
+            // experts find each other with match_any, 32 pairs at a time.
+            constexpr int EPL = 8;
+            const int np = T * K;
+            const uint32_t lt = (1u << lane) - 1u;
+            for (int q = lane; q < kMaxActive; q += 32) s_off[q] = 0;   // histogram first
+            __syncwarp();
+            int prow[2];
+            for (int h = 0; h < 2; ++h) {
+                const int p = 32 * h + lane;
+                const int e = p < np ? s_sel[p] : E + lane;   // lanes without a pair match nobody real
+                const uint32_t m = __match_any_sync(0xFFFFFFFFu, e);
+                prow[h] = (p < np ? s_off[e] : 0) + __popc(m & lt);
+                __syncwarp();
+                if (p < np && (m & lt) == 0) s_off[e] += __popc(m);   // the group's first lane counts it
+                __syncwarp();
+            }
+            int cnt[EPL], mine = 0, tot = 0;
+#pragma unroll
+            for (int q = 0; q < EPL; ++q) {
+                const int e = lane * EPL + q;
+                cnt[q] = e < E ? s_off[e] : 0;
+                tot += cnt[q];
+                mine += cnt[q] > 0;
+            }
+            __syncwarp();
+            int incl = tot, incl_act = mine;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+                const int oa = __shfl_up_sync(0xFFFFFFFFu, incl_act, off);
+                if (lane >= off) {
+                    incl += o;
+                    incl_act += oa;
+                }
+            }
+            int run = incl - tot;
+            const int first = a.has_shared ? 1 : 0;
+            int slot = first + incl_act - mine;
+#pragma unroll
+            for (int q = 0; q < EPL; ++q) {
+                const int e = lane * EPL + q;
+                if (e < E) {
+                    s_off[e] = run;
+                    if (blockIdx.x == 0) {
+                        ga.r.offsets[e] = run;
+                        ga.r.counts[e] = cnt[q];
+                    }
+                }
+                if (cnt[q] > 0) {
+                    act_e[slot] = e;
+                    act_row0[slot] = run;
+                    act_cnt[slot] = cnt[q];
+                    ++slot;
+                }
+                run += cnt[q];
+            }
+            if (lane == 31) {
+                if (a.has_shared) {
+                    act_e[0] = E;
+                    act_row0[0] = 0;
+                    act_cnt[0] = T;
+                }
+                s_misc[0] = first + incl_act;
+                if (blockIdx.x == 0) ga.r.offsets[E] = incl;
+            }
+            __syncwarp();
+            for (int h = 0; h < 2; ++h) {
+                const int p = 32 * h + lane;
+                if (p < np) {
+                    const int e = s_sel[p];
+                    const int row = s_off[e] + prow[h];
+                    s_r2p[row] = p;
+                    s_pw[p] = s_selw[p];
+                    if (blockIdx.x == 0) {
+                        ga.r.row_to_pair[row] = p;
+                        ga.r.pair_to_row[p] = row;
+                        ga.r.topk_idx[p] = e;
+                        ga.r.topk_w[p] = s_selw[p];
+                    }
+                }
+            }
+            __syncwarp();
+            __threadfence_block();
+            named_barrier_arrive(8, kThreads);
+            const int A = s_misc[0];
+            if (lane == 0) {
+                int k = 0;
+                for (int u = blockIdx.x; u < A * NJ; u += gridDim.x, ++k) {
+                    if (k == 0 && early) continue;
+                    issue_unit(k, act_e[u / NJ], u % NJ);
+                }
+            }
+            __syncwarp();
+        }
+    } else if (warp == kConsumerWarps) {
         // ---- active experts (the shared one first, then routed ones with rows)
         constexpr int EPL = 8;   // experts per lane (E <= 256)
         int ofs[EPL + 1];
@@ -311,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int jr = 8 * t + perm8(g);               // gate/up row (of the unit's 32) of MMA rows g, g+8
         const int TW = H / 256;                        // 16-row down tiles per warp
         const int nbase = 16 * TW * warp;              // first down row of this warp
-        bool zero_seen = false;
+        bool zero_seen = kRoute;   // the routing barrier already covered the zeroing
         int k = 0;
         for (int u = blockIdx.x; u < A * NJ; u += gridDim.x, ++k) {
             const int ai = u / NJ, jb = u % NJ;
@@ -543,21 +771,21 @@ bool ffn_gemv_supported(const FfnArgs& a) {
            (a.H == 512 || a.H == 1024 || a.H == 2048) && a.I % 64 == 0 && a.I >= 64 && a.I <= 8192;
 }
 
-cudaError_t launch_ffn_gemv(const FfnArgs& a, unsigned long long* sync, cudaStream_t st) {
-    GemvArgs ga;
-    ga.f = a;
-    ga.L = gemv_layout(a.H);
-    ga.sync = sync;
+namespace {
+
+template <bool kRoute>
+cudaError_t launch_gemv(const GemvArgs& ga, cudaStream_t st) {
     CUtensorMap gu_map, d_map;
-    if (!make_gu_map(&gu_map, a) || !make_d_map(&d_map, a)) return cudaErrorInvalidValue;
+    if (!make_gu_map(&gu_map, ga.f) || !make_d_map(&d_map, ga.f)) return cudaErrorInvalidValue;
     static int done[64] = {0};
     const int smem = ga.L.total + 1024;
-    cudaError_t ce = set_smem_once(k_ffn_gemv, smem, done);
+    cudaError_t ce = set_smem_once(k_ffn_gemv<kRoute>, smem, done);
     if (ce != cudaSuccess) return ce;
     const int G = num_sms_cached();
     if (G <= 0) return cudaErrorInvalidDevice;
-    // one CTA per SM, all resident at once (the in-kernel count of zeroing
-    // CTAs waits for every CTA of the launch)
+    if (kRoute && G * kConsumerWarps < ga.f.E) return cudaErrorInvalidConfiguration;
+    // one CTA per SM, all resident at once (the in-kernel counts wait for
+    // every CTA of the launch)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(G);
     cfg.blockDim = dim3(kThreads);
@@ -568,7 +796,39 @@ cudaError_t launch_ffn_gemv(const FfnArgs& a, unsigned long long* sync, cudaStre
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_ffn_gemv, gu_map, d_map, ga);
+    return cudaLaunchKernelEx(&cfg, k_ffn_gemv<kRoute>, gu_map, d_map, ga);
+}
+
+}  // namespace
+
+cudaError_t launch_ffn_gemv(const FfnArgs& a, unsigned long long* sync, cudaStream_t st) {
+    GemvArgs ga = {};
+    ga.f = a;
+    ga.L = gemv_layout(a.H);
+    ga.sync = sync;
+    return launch_gemv<false>(ga, st);
+}
+
+bool decode_fused_supported(const FfnArgs& a) {
+    return ffn_gemv_supported(a) && a.E == 256 && a.H <= 2048;
+}
+
+cudaError_t launch_decode_fused(const FfnArgs& a, const DecodeRoute& r, unsigned long long* sync, cudaStream_t st) {
+    GemvArgs ga = {};
+    ga.f = a;
+    ga.L = gemv_layout(a.H);
+    ga.sync = sync;
+    ga.r.w_router = r.w_router;
+    ga.r.bias = r.bias;
+    ga.r.bias_stride = r.bias_stride;
+    ga.r.logits = r.logits;
+    ga.r.topk_idx = r.topk_idx;
+    ga.r.topk_w = r.topk_w;
+    ga.r.counts = r.counts;
+    ga.r.offsets = r.offsets;
+    ga.r.row_to_pair = r.row_to_pair;
+    ga.r.pair_to_row = r.pair_to_row;
+    return launch_gemv<true>(ga, st);
 }
 
 }  // namespace moe

@@ -70,6 +70,24 @@ cudaError_t launch_ffn_simt(const FfnArgs& a, cudaStream_t st);
 bool ffn_gemv_supported(const FfnArgs& a);
 cudaError_t launch_ffn_gemv(const FfnArgs& a, unsigned long long* sync, cudaStream_t st);
 cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st);
+
+// Decode layer in one kernel: router logits, top-k, permutation and expert
+// FFN (scatter into y_acc); the routing outputs are written as the route and
+// permute calls would.
+struct DecodeRoute {
+    const uint16_t* w_router;
+    const float* bias;
+    int64_t bias_stride;
+    float* logits;
+    int32_t* topk_idx;
+    float* topk_w;
+    int32_t* counts;
+    int32_t* offsets;
+    int32_t* row_to_pair;
+    int32_t* pair_to_row;
+};
+bool decode_fused_supported(const FfnArgs& a);
+cudaError_t launch_decode_fused(const FfnArgs& a, const DecodeRoute& r, unsigned long long* sync, cudaStream_t st);
 bool ffn_tc_supported(const FfnArgs& a);
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st);
 

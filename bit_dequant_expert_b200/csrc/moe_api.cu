@@ -243,6 +243,62 @@ int32_t moe_get_device_error(const void* ws, void* stream) {
     return v;
 }
 
+int32_t moe_decode_layer(const moe_config_t* cfg, int32_t T, const uint16_t* x, const uint16_t* w_router,
+                         const float* logit_bias, int64_t logit_bias_row_stride, const uint32_t* gu_codes,
+                         const uint16_t* gu_sb, const uint32_t* d_codes, const uint16_t* d_sb, int32_t* topk_idx,
+                         float* topk_w, int32_t* counts, int32_t* offsets, int32_t* row_to_pair,
+                         int32_t* pair_to_row, float* y_acc, uint16_t* y, void* ws, size_t ws_bytes,
+                         void* stream) {
+    if (!ws) return MOE_ERR_WORKSPACE;
+    int32_t st = check_common(cfg, T, ws, ws_bytes);
+    if (st) return st;
+    if (!x || !w_router || !gu_codes || !gu_sb || !d_codes || !d_sb || !topk_idx || !topk_w || !counts ||
+        !offsets || !row_to_pair || !pair_to_row || !y_acc || !y)
+        return MOE_ERR_INVALID_ARG;
+    if (logit_bias_row_stride < 0) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(logit_bias, 4) || !aligned(gu_codes, 256) ||
+        !aligned(gu_sb, 256) || !aligned(d_codes, 256) || !aligned(d_sb, 256) || !aligned(topk_idx, 4) ||
+        !aligned(topk_w, 4) || !aligned(counts, 4) || !aligned(offsets, 4) || !aligned(row_to_pair, 4) ||
+        !aligned(pair_to_row, 4) || !aligned(y_acc, 16) || !aligned(y, 16))
+        return MOE_ERR_INVALID_ARG;
+    FfnArgs a = shape_only(cfg, T);
+    a.mode = MOE_MODE_SCATTER;
+    if (!decode_fused_supported(a)) return MOE_ERR_UNSUPPORTED;
+    a.x = x;
+    a.gu_codes = gu_codes;
+    a.gu_sb = gu_sb;
+    a.d_codes = d_codes;
+    a.d_sb = d_sb;
+    a.offsets = offsets;
+    a.row_to_pair = row_to_pair;
+    a.topk_w = topk_w;
+    a.y_acc = y_acc;
+    a.err = err_word(ws);
+    DecodeRoute r;
+    r.w_router = w_router;
+    r.bias = logit_bias;
+    r.bias_stride = logit_bias_row_stride;
+    r.logits = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + layout(cfg, T).logits);
+    r.topk_idx = topk_idx;
+    r.topk_w = topk_w;
+    r.counts = counts;
+    r.offsets = offsets;
+    r.row_to_pair = row_to_pair;
+    r.pair_to_row = pair_to_row;
+    cudaStream_t s = (cudaStream_t)stream;
+    st = cuda_status(launch_decode_fused(a, r, &reinterpret_cast<WsHeader*>(ws)->grid_sync, s));
+    if (st) return st;
+    CombineArgs c = {};
+    c.T = T;
+    c.H = cfg->hidden;
+    c.has_shared = cfg->has_shared;
+    c.mode = MOE_MODE_SCATTER;
+    c.y_acc = y_acc;
+    c.y = y;
+    c.err = err_word(ws);
+    return cuda_status(launch_combine(c, s));
+}
+
 int32_t moe_launch_count(const moe_config_t* cfg, int32_t T, int32_t mode, int32_t path) {
     if (!config_ok(cfg) || T < 1 || T > kMaxTokens) return -1;
     if (mode != MOE_MODE_SCATTER && mode != MOE_MODE_PAIRS) return -1;

@@ -169,8 +169,8 @@ __global__ void __launch_bounds__(256) k_perm_small(int T, int E, const int32_t*
                                                     int32_t* __restrict__ pair_to_row, int32_t* err) {
     extern __shared__ uint32_t mask[];
     int* s_off = reinterpret_cast<int*>(mask + E * (kChunk / 32));
-    griddep_wait();   // idx and counts come from the router
-    griddep_launch_dependents();
+    griddep_launch_dependents();   // the next grid may start its own prologue
+    griddep_wait();                // idx and counts come from the router
     build_masks<K>(T, E, 0, idx, mask, err);
     // E <= 1024: each thread scans E / blockDim.x experts in order
     const int per = (E + blockDim.x - 1) / blockDim.x;

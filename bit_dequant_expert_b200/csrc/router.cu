@@ -9,6 +9,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
+#include "topk.cuh"
 
 namespace moe {
 
@@ -99,90 +100,6 @@ __global__ void __launch_bounds__(256) k_router_logits(int T, int H, int E, cons
     router_tile<TT, TE>(T, H, E, blockIdx.x * TT, (blockIdx.y * 8 + warp) * TE, x, wr, bias, bias_stride, logits);
 }
 
-// Order-preserving map of a finite float to uint32 (larger float -> larger
-// key); -0.0 is folded onto +0.0 so the two tie.
-__device__ __forceinline__ uint32_t order_key(float f) {
-    if (f == 0.0f) f = 0.0f;
-    const uint32_t u = __float_as_uint(f);
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-__device__ __forceinline__ float key_value(uint32_t k) {
-    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
-}
-
-// One warp per token.  Lane l holds the logits of experts l, l+32, ...; each
-// of the K rounds takes the warp-wide maximum of (value, -index) and retires
-// the winner.  Weights are the softmax over the K selected logits, which is
-// the E-way softmax restricted to them and renormalised.
-template <int EPL, int K>
-__device__ __forceinline__ void topk_token(int t, int E, const float* __restrict__ logits,
-                                           const float* __restrict__ bias, int64_t bias_stride,
-                                           int32_t* __restrict__ idx, float* __restrict__ wout,
-                                           int32_t* __restrict__ counts, int32_t* err) {
-    const int lane = threadIdx.x & 31;
-    float v[EPL];
-    bool bad = false;
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-        const int e = lane + 32 * i;
-        float l = __ldcg(logits + (size_t)t * E + e);
-        if (bias) l = __fadd_rn(l, bias[(int64_t)t * bias_stride + e]);
-        v[i] = l;
-        bad |= !isfinite(l);
-    }
-    if (__any_sync(0xFFFFFFFFu, bad)) {
-        if (lane == 0) set_error(err, MOE_ERR_NONFINITE);
-        if (lane < K) {
-            idx[(size_t)t * K + lane] = lane;
-            wout[(size_t)t * K + lane] = 1.0f / K;
-            atomicAdd(&counts[lane], 1);
-        }
-        return;
-    }
-    uint32_t key[EPL];
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) key[i] = order_key(v[i]);
-    uint32_t taken = 0;
-    int sel_e[K];
-    float sel_v[K];
-#pragma unroll
-    for (int r = 0; r < K; ++r) {
-        unsigned long long best = 0ull;
-#pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-            const unsigned long long kk =
-                ((unsigned long long)key[i] << 32) | (uint32_t)(~(uint32_t)(lane + 32 * i));
-            if (!((taken >> i) & 1u) && kk > best) best = kk;
-        }
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) {
-            const unsigned long long o = __shfl_xor_sync(0xFFFFFFFFu, best, off);
-            best = o > best ? o : best;
-        }
-        const int e = (int)(~(uint32_t)best);
-        if ((e & 31) == lane) taken |= 1u << (e >> 5);
-        sel_e[r] = e;
-        sel_v[r] = key_value((uint32_t)(best >> 32));
-    }
-    const float m = sel_v[0];
-    float ex[K];
-    float s = 0.0f;
-#pragma unroll
-    for (int r = 0; r < K; ++r) {
-        ex[r] = expf(sel_v[r] - m);
-        s += ex[r];
-    }
-#pragma unroll
-    for (int r = 0; r < K; ++r) {
-        if (lane == r) {
-            idx[(size_t)t * K + r] = sel_e[r];
-            wout[(size_t)t * K + r] = ex[r] / s;
-            atomicAdd(&counts[sel_e[r]], 1);
-        }
-    }
-}
-
 template <int EPL, int K>
 __global__ void __launch_bounds__(256) k_topk(int T, int E, const float* __restrict__ logits,
                                               const float* __restrict__ bias, int64_t bias_stride,
@@ -243,8 +160,8 @@ __global__ void __launch_bounds__(64) k_route_small_wide(int T, int H, int E, co
         const int c = lane + 32 * i;
         wv[i] = c < nchunk ? ldg_v4(wr + (size_t)e * H + 8 * c) : make_uint4(0, 0, 0, 0);
     }
-    griddep_wait();
-    griddep_launch_dependents();
+    griddep_launch_dependents();   // the next grid may start its own prologue
+    griddep_wait();                // x may come from the previous grid
     for (int q = threadIdx.x; q < T * nchunk; q += blockDim.x) xs4[q] = reinterpret_cast<const uint4*>(x)[q];
     __syncthreads();
     float acc[8];

@@ -6,8 +6,8 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (MOE_MODE_PAIRS, MOE_MODE_SCATTER, MOE_PATH_AUTO, config, moe_combine, moe_expert_ffn_path,
-               moe_permute, moe_route, moe_workspace_init, moe_workspace_size)
+from . import (MOE_MODE_PAIRS, MOE_MODE_SCATTER, MOE_PATH_AUTO, config, moe_combine, moe_decode_layer,
+               moe_expert_ffn_path, moe_permute, moe_route, moe_workspace_init, moe_workspace_size)
 
 
 def to_device(a, device, dtype=None) -> torch.Tensor:
@@ -97,8 +97,23 @@ class MoELayer:
         T = x.shape[0]
         if T > self.max_tokens:
             raise ValueError("T=%d exceeds max_tokens=%d" % (T, self.max_tokens))
+        if self.fused_ok(T) and logits_in is None:
+            return self.decode_fused(x, T, logit_bias, bias_stride, stream, y_out)
         self.route(x, T, logit_bias, bias_stride, logits_in, stream)
         self.permute(T, stream)
         self.expert_ffn(x, T, stream)
         self.combine(T, stream, y_out)
+        return self.y[:T] if y_out is None else y_out
+
+    def fused_ok(self, T) -> bool:
+        """Whether forward() takes the two-launch decode layer for T tokens."""
+        return (T <= 8 and self.mode == MOE_MODE_SCATTER and self.path == MOE_PATH_AUTO and self.E == 256
+                and self.H in (512, 1024, 2048))
+
+    def decode_fused(self, x, T, logit_bias=None, bias_stride=0, stream=None, y_out=None) -> torch.Tensor:
+        """The layer for T <= 8 tokens in two launches (moe_decode_layer)."""
+        y = self.y if y_out is None else y_out
+        moe_decode_layer(self.cfg, T, x, self.w_router, logit_bias, bias_stride, self.gu_codes, self.gu_sb,
+                         self.d_codes, self.d_sb, self.topk_idx, self.topk_w, self.counts, self.offsets,
+                         self.row_to_pair, self.pair_to_row, self.out0, y, self.ws, stream=stream)
         return self.y[:T] if y_out is None else y_out

@@ -176,6 +176,30 @@ int32_t moe_expert_ffn_path(const moe_config_t* cfg, int32_t T, const uint16_t* 
 int32_t moe_combine(const moe_config_t* cfg, int32_t T, int32_t mode, const void* in0, const void* in1,
                     const int32_t* pair_to_row, const float* topk_w, uint16_t* y, void* stream);
 
+/*
+ * moe_decode_layer: the whole layer for a handful of tokens in two launches
+ * (decode-step integration).  Computes exactly what moe_route (x, w_router,
+ * optional logit bias; logits computed by the router, not given) ->
+ * moe_permute -> moe_expert_ffn (MOE_MODE_SCATTER) -> moe_combine compute,
+ * and writes every intermediate those calls write: topk_idx, topk_w, counts,
+ * offsets, row_to_pair, pair_to_row, y_acc fp32 [T, H] and y bf16 [T, H].
+ * Lily pages: "Perplexity built an inference engine for one model, one
+ * chip", third paragraph (the routing decision stays on the GPU with the
+ * expert work; the decode step as few kernels as possible).
+ * The first kernel computes the router logits over all CTAs, meets at a
+ * grid-wide (bounded) barrier, selects the top-k and builds the permutation
+ * in every CTA, then runs the decode expert FFN; the second converts y_acc.
+ * Supported: 1 <= T <= 8, hidden 512, 1024 or 2048, E == 256, k == 8;
+ * otherwise MOE_ERR_UNSUPPORTED before any launch (use the four calls).
+ * Same pointer rules as the four calls; the workspace must hold T tokens.
+ */
+int32_t moe_decode_layer(const moe_config_t* cfg, int32_t T, const uint16_t* x, const uint16_t* w_router,
+                         const float* logit_bias, int64_t logit_bias_row_stride, const uint32_t* gu_codes,
+                         const uint16_t* gu_sb, const uint32_t* d_codes, const uint16_t* d_sb, int32_t* topk_idx,
+                         float* topk_w, int32_t* counts, int32_t* offsets, int32_t* row_to_pair,
+                         int32_t* pair_to_row, float* y_acc, uint16_t* y, void* ws, size_t ws_bytes,
+                         void* stream);
+
 /* Synchronises `stream` and returns the workspace's sticky device error
  * (MOE_OK if none), or MOE_ERR_CUDA if the synchronisation failed. */
 int32_t moe_get_device_error(const void* ws, void* stream);

@@ -80,3 +80,24 @@ def test_host_validation_before_launch():
     assert st == m.MOE_ERR_INVALID_ARG
     assert m.moe_get_device_error(None, 0) == m.MOE_ERR_WORKSPACE
     assert m.moe_status_string(m.MOE_ERR_NONFINITE) == "MOE_ERR_NONFINITE"
+
+
+def _decode(cfg, T, ws_bytes, x=FAKE, y=FAKE, bias=None, stride=0):
+    import bit_dequant_expert_b200 as m
+    return m.moe_decode_layer(cfg, T, x, FAKE, bias, stride, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                              FAKE, FAKE, y, FAKE, ws_bytes=ws_bytes, stream=0, raise_on_error=False)
+
+
+def test_decode_layer_validation_before_launch():
+    """The fused decode call takes 1 <= T <= 8 at hidden 512/1024/2048; anything
+    else, a bad pointer or a short workspace is refused before any launch."""
+    import bit_dequant_expert_b200 as m
+    cfg = m.config()
+    need = m.moe_workspace_size(cfg, 16)
+    assert _decode(cfg, 9, need) == m.MOE_ERR_UNSUPPORTED
+    assert _decode(m.config(hidden=4096), 1, m.moe_workspace_size(m.config(hidden=4096), 1)) == m.MOE_ERR_UNSUPPORTED
+    assert _decode(cfg, 0, need) == m.MOE_ERR_INVALID_ARG
+    assert _decode(cfg, 8, 256) == m.MOE_ERR_WORKSPACE
+    assert _decode(cfg, 8, need, x=None) == m.MOE_ERR_INVALID_ARG
+    assert _decode(cfg, 8, need, y=FAKE + 8) == m.MOE_ERR_INVALID_ARG
+    assert _decode(cfg, 8, need, bias=FAKE, stride=-1) == m.MOE_ERR_INVALID_ARG

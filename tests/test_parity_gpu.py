@@ -260,6 +260,97 @@ def test_gemv_all_tokens_same_experts():
     check_output(out, lay, np.arange(8))
 
 
+# ------------------------------------------------------------ fused decode layer (moe_decode_layer)
+
+AUTO = 0
+
+
+def _fused_vs_oracle(lay, T):
+    out, L = run_layer(lay, SCATTER, AUTO)
+    assert L.fused_ok(T)
+    assert out["err"] == 0
+    idx_ref = check_routing(out, lay)
+    counts, offsets, r2p, p2r = oracle.permute(idx_ref, 256)
+    assert np.array_equal(out["counts"], counts) and np.array_equal(out["offsets"], offsets)
+    assert np.array_equal(out["r2p"], r2p) and np.array_equal(out["p2r"], p2r)
+    check_output(out, lay, np.arange(T))
+    return out, L
+
+
+@pytest.mark.parametrize("T", [1, 2, 5, 8])
+def test_fused_decode_small_shapes(T):
+    _fused_vs_oracle(layer_of(0, T=T), T)
+
+
+def test_fused_decode_layers():
+    spec = gen.config(1)
+    for layer in (0, 21, 39):
+        _fused_vs_oracle(gen.make_layer(spec, layer), 1)
+
+
+@pytest.mark.parametrize("T", [1, 7])
+def test_fused_decode_hidden_1024(T):
+    spec = gen.LayerSpec(T=T, H=1024, I=256, seed=12)
+    _fused_vs_oracle(gen.make_layer(spec, 0), T)
+
+
+@pytest.mark.parametrize("per_token", [False, True])
+def test_fused_decode_logit_bias(per_token):
+    lay = dict(layer_of(0, T=6))
+    rng = np.random.default_rng(5)
+    if per_token:
+        lay["logit_bias"] = (rng.standard_normal((6, 256)) * 0.05).astype(np.float32)
+        lay["bias_stride"] = 256
+    else:
+        bias = np.zeros(256, dtype=np.float32)
+        bias[[4, 8, 15, 16, 23, 42, 99, 255]] = 100.0   # every token picks the same eight
+        lay["logit_bias"], lay["bias_stride"] = bias, 0
+    out, _ = _fused_vs_oracle(lay, 6)
+    if not per_token:
+        assert np.all(np.sort(out["idx"], axis=1) == [4, 8, 15, 16, 23, 42, 99, 255])
+
+
+def test_fused_decode_matches_four_calls_and_repeats():
+    """Routing outputs are identical to the four calls'; repeated calls (which
+    reuse the grid barrier counter) stay correct."""
+    import torch
+    from bit_dequant_expert_b200.layer import MoELayer, to_device
+    lay = layer_of(3, T=8)
+    Lf = MoELayer(lay, max_tokens=8, mode=SCATTER)
+    Lg = MoELayer(lay, max_tokens=8, mode=SCATTER, path=GEMV)
+    x = to_device(lay["x"], "cuda")
+    yg = Lg.forward(x).float().cpu().numpy()
+    first = Lf.forward(x).float().cpu().numpy().copy()
+    for name in ("topk_idx", "topk_w", "counts", "offsets", "row_to_pair", "pair_to_row"):
+        assert torch.equal(getattr(Lf, name), getattr(Lg, name)), name
+    for _ in range(5):
+        again = Lf.forward(x).float().cpu().numpy()
+        assert np.max(row_rel_err(again.astype(np.float64), first.astype(np.float64))) < 1e-2
+    import bit_dequant_expert_b200 as m
+    assert m.moe_get_device_error(Lf.ws) == 0
+    assert np.max(row_rel_err(first.astype(np.float64), yg.astype(np.float64))) < 1e-2
+
+
+def test_fused_decode_nonfinite_input_sets_error():
+    import bit_dequant_expert_b200 as m
+    lay = dict(layer_of(0, T=2))
+    x = lay["x"].copy()
+    x[1, 10] = 0x7FC0          # bf16 NaN: every logit of token 1 is NaN
+    lay["x"] = x
+    out, L = run_layer(lay, SCATTER, AUTO)
+    assert L.fused_ok(2)
+    assert out["err"] == m.MOE_ERR_NONFINITE
+    assert out["idx"][1].tolist() == list(range(8)) and np.all(out["w"][1] == 0.125)
+
+
+def test_fused_decode_unsupported_shapes_fall_back():
+    lay = layer_of(0, T=9)
+    out, L = run_layer(lay, SCATTER, AUTO)
+    assert not L.fused_ok(9)
+    assert out["err"] == 0
+    check_output(out, lay, np.arange(9))
+
+
 # ------------------------------------------------------------ tensor-core (tcgen05) path
 
 
