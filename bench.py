@@ -367,6 +367,32 @@ def run_prefill(device, steps, warmup, world, peaks):
             "l2": "inputs larger than L2 (455.8 MB of packed weights per layer)"}
 
 
+def run_ncu_case(case, device, calls):
+    """One layer for a profiler: route + permute, then `calls` launches of the kernel under study."""
+    import torch
+    import gen
+    import bit_dequant_expert_b200 as m
+    from bit_dequant_expert_b200 import MOE_MODE_PAIRS, MOE_MODE_SCATTER
+    from bit_dequant_expert_b200.layer import MoELayer, to_device
+    spec = gen.config(3 if case == "prefill-ffn" else 1)
+    lay = gen.make_layer(spec, 0)
+    T = spec.T
+    L = MoELayer(lay, max_tokens=T, device=device,
+                 mode=MOE_MODE_PAIRS if case == "prefill-ffn" else MOE_MODE_SCATTER)
+    x = to_device(lay["x"], device)
+    del lay
+    L.route(x, T)
+    L.permute(T)
+    for _ in range(calls):
+        if case == "decode-layer":
+            L.forward(x)
+        else:
+            L.expert_ffn(x, T)
+    torch.cuda.synchronize()
+    print(json.dumps({"ncu_case": case, "calls": calls, "device_error": m.moe_get_device_error(L.ws)}))
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -376,6 +402,10 @@ def main(argv=None):
     ap.add_argument("--no-prefill", action="store_true", help="skip the T=2048 prefill measurement")
     ap.add_argument("--prefill-only", action="store_true",
                     help="measure only the T=2048 prefill layer (its line replaces the decode line)")
+    ap.add_argument("--ncu-case", choices=("decode-ffn", "decode-layer", "prefill-ffn"),
+                    help="a small case for a profiler capture: one synthetic layer, route + permute, then "
+                         "--steps calls of the named kernel (decode: config 1 layer 0, T=1; prefill: "
+                         "config 3, T=2048); prints the device error word and nothing timed")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle CPU baseline")
     args = ap.parse_args(argv)
     warmup = max(args.warmup, 3)
@@ -392,6 +422,9 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     device = torch.device("cuda", torch.cuda.current_device())
     peaks = load_peaks()
+
+    if args.ncu_case:
+        return run_ncu_case(args.ncu_case, device, max(args.steps, 1))
 
     if args.prefill_only:
         pre = run_prefill(device, max(args.steps, 1), warmup, world, peaks)
