@@ -41,11 +41,11 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kNT = 128;                 // token rows per tile (MMA N, max)
 static_assert(kNT % 64 == 0, "the column-table builders cover kNT columns with 64 threads");
-constexpr int kBK = 64;                  // inputs per chunk = one (scale, bias) group
-constexpr int kStages = 6;              // B ring and TMEM A stages (64 inputs each)
+constexpr int kBK = 128;                 // inputs per chunk = two (scale, bias) groups
+constexpr int kStages = 3;              // B ring and TMEM A stages (128 inputs each)
 constexpr int kCStages = 4;             // codes ring
 constexpr int kCodesStage = 128 * 128;  // 128 rows x 256 nibbles (four chunks), 128B-swizzled
-constexpr int kBStage = kNT * 128;       // kNT rows x 64 bf16
+constexpr int kBStage = kNT * 2 * 128;   // two 64-input halves of kNT rows x 64 bf16
 constexpr int kACol0 = 2 * kNT;          // TMEM: two fp32 accumulators, then the A stages
 constexpr int kAStageCols = kBK / 2;     // bf16 pairs per 32-bit column
 constexpr int kTmemCols = 512;
@@ -155,8 +155,9 @@ __device__ __forceinline__ int wrow_up(const FfnArgs& a, const Tile& tl) { retur
 __device__ __forceinline__ int wrow_down(const FfnArgs& a, const Tile& tl) { return tl.e * a.H + 128 * tl.mb; }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    k_ffn_tc(const __grid_constant__ CUtensorMap codes_map, const __grid_constant__ CUtensorMap b_map,
-             const __grid_constant__ CUtensorMap sb_map, const TcArgs ta) {
+    k_ffn_tc(const __grid_constant__ CUtensorMap codes_map, const __grid_constant__ CUtensorMap b_map64,
+             const __grid_constant__ CUtensorMap b_map128, const __grid_constant__ CUtensorMap sb_map,
+             const TcArgs ta) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // the 128B-swizzled B stages need a 1024-byte aligned base
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -169,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // codes come in stages of cw u32 words (8 cw inputs) per row: 256 inputs,
     // or all of K when K is shorter; a stage feeds cps chunks
     const int cw = K >= 256 ? 32 : K / 8;
-    const int cps = cw / 8;
+    const int cps = cw / 16;
     // (scale, bias) rows go through shared memory by TMA when a row's words
     // span whole 16-byte units; otherwise (tiny K) each thread reads its own
     const bool sb_tma = (ngroups & 3) == 0;
@@ -242,10 +243,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (cit >= kCStages) mbar_wait_bounded(&sm.cempty[cs], ((cit / kCStages) - 1) & 1, a.err);
                         mbar_arrive_expect_tx(&sm.cfull[cs], 128 * cw * 4);
                         if (gateup) {
-                            tma_load_2d(sm.codes[cs], &codes_map, kc * 8, wrow_gate(a, tl), &sm.cfull[cs]);
-                            tma_load_2d(sm.codes[cs] + 64 * cw * 4, &codes_map, kc * 8, wrow_up(a, tl), &sm.cfull[cs]);
+                            tma_load_2d(sm.codes[cs], &codes_map, kc * 16, wrow_gate(a, tl), &sm.cfull[cs]);
+                            tma_load_2d(sm.codes[cs] + 64 * cw * 4, &codes_map, kc * 16, wrow_up(a, tl), &sm.cfull[cs]);
                         } else {
-                            tma_load_2d(sm.codes[cs], &codes_map, kc * 8, wrow_down(a, tl), &sm.cfull[cs]);
+                            tma_load_2d(sm.codes[cs], &codes_map, kc * 16, wrow_down(a, tl), &sm.cfull[cs]);
                         }
                     }
                 }
@@ -269,11 +270,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_wait_bounded(&sm.a_full[s], par, a.err);
                     mbar_wait_bounded(&sm.full[s], par, a.err);
                     tc_fence_after();
-                    const uint64_t bdesc = smem_desc_sw128(smem_u32(sm.b[s]));
+                    // B stage: two 64-input halves of R token rows each (R = 64 or 128)
+                    const int R = tl.npad > 64 ? 128 : 64;
+                    const uint64_t bdesc0 = smem_desc_sw128(smem_u32(sm.b[s]));
+                    const uint64_t bdesc1 = smem_desc_sw128(smem_u32(sm.b[s] + R * 128));
                     const uint32_t a_tmem = tmem + kACol0 + s * kAStageCols;
 #pragma unroll
                     for (int j = 0; j < kBK / 16; ++j)
-                        tc_mma_ts(d_tmem, a_tmem + 8 * j, bdesc + 2 * j, idesc, (kc | j) != 0);
+                        tc_mma_ts(d_tmem, a_tmem + 8 * j, (j < 4 ? bdesc0 : bdesc1) + 2 * (j & 3), idesc,
+                                  (kc | j) != 0);
                     tc_commit(&sm.mma_done[s]);
                 }
                 tc_commit(&sm.acc_full[ab]);
@@ -316,15 +321,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.tab_full[slot]);
             }
-            const int nbox = tl.npad > 64 ? 2 : 1;   // 64-row boxes
+            // one 3-D box per chunk: R token rows x two 64-input halves
+            const int R = tl.npad > 64 ? 128 : 64;
             for (int kc = 0; kc < KC; ++kc, ++it) {
                 if ((it & 1u) != par) continue;
                 const int s = it % kStages;
                 if (lane == 0) {
                     if (it >= kStages) mbar_wait_bounded(&sm.mma_done[s], ((it / kStages) - 1) & 1, a.err);
-                    mbar_arrive_expect_tx(&sm.full[s], nbox * 64 * 128);
-                    for (int bx = 0; bx < nbox; ++bx)
-                        tma_load_2d(sm.b[s] + bx * 64 * 128, &b_map, kc * kBK, (int)tl.hrow0 + 64 * bx, &sm.full[s]);
+                    mbar_arrive_expect_tx(&sm.full[s], R * 2 * 128);
+                    tma_load_3d(sm.b[s], R == 128 ? &b_map128 : &b_map64, 0, (int)tl.hrow0, 2 * kc, &sm.full[s]);
                 }
                 __syncwarp();
             }
@@ -332,18 +337,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp < 12) {
         // ------------------------------------------------------------ dequantisers
         const int q = warp & 3;              // TMEM lane quadrant
-        const int khalf = (warp - 4) >> 2;   // which 32 inputs of the chunk
+        const int khalf = (warp - 4) >> 2;   // which 64 inputs (group) of the chunk
         const int L = 32 * q + lane;         // A row == TMEM lane
-        const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16) + kACol0 + 16 * khalf;
+        const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16) + kACol0 + 32 * khalf;
         const uint32_t* sbase = reinterpret_cast<const uint32_t*>(gateup ? a.gu_sb : a.d_sb);
         // codes of row L inside a stage: gate/up interleave gate and up rows on
         // adjacent lanes (even: gate, odd: up), so SwiGLU pairs are lane pairs
         // row of lane L inside a codes stage; rows are cw words wide and, when
         // 128 bytes wide, 128B-swizzled (16-byte unit u of row r sits at u ^ (r & 7))
         const int crow = gateup ? ((L & 1) * 64 + (L >> 1)) : L;
-        auto codes_at = [&](int cs, int kc) -> uint4 {
-            const int unit = (kc % cps) * 2 + khalf;
-            const int phys = cw == 32 ? (unit ^ (crow & 7)) : unit;
+        // 16-byte unit u of row crow in codes stage cs (128B-swizzled when the rows are
+        // 128 bytes wide: unit u of row r sits at u ^ (r & 7))
+        auto codes_at = [&](int cs, int u) -> uint4 {
+            const int phys = cw == 32 ? (u ^ (crow & 7)) : u;
             return *reinterpret_cast<const uint4*>(sm.codes[cs] + crow * cw * 4 + phys * 16);
         };
         uint32_t it = 0, lt = 0;
@@ -355,56 +361,47 @@ __global__ void __launch_bounds__(kThreads, 1)
             // this row's (scale, bias) words in shared memory: gate rows 0..63, up rows 64..127
             const uint32_t* sbs_row = sm.sbs[buf] + (size_t)(gateup ? ((L & 1) * 64 + (L >> 1)) : L) * ngroups;
             if (sb_tma) mbar_wait_bounded(&sm.sb_full[buf], (lt >> 1) & 1, a.err);
-            uint4 cur = make_uint4(0, 0, 0, 0);
-            auto sb_of = [&](int kc) -> uint32_t {
-                if (!sb_tma) return ldg_u32(sbrow + kc);
-                const int r = kc & 3;
-                if (r == 0) cur = *reinterpret_cast<const uint4*>(sbs_row + kc);
-                return r == 0 ? cur.x : r == 1 ? cur.y : r == 2 ? cur.z : cur.w;
-            };
-            auto dequant16 = [&](uint4 cw, uint32_t sbw, uint32_t (&v)[16]) {
+            auto dequant16 = [&](uint4 cw, uint32_t sbw, uint32_t* v) {
                 const uint32_t s2 = prmt(sbw, sbw, 0x1010), b2 = prmt(sbw, sbw, 0x3232);
                 const uint32_t wds[4] = {cw.x, cw.y, cw.z, cw.w};
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
                     const uint32_t w0 = wds[m], w4 = w0 >> 4;
-                    v[4 * m + 0] = dequant_pair<0>(w0, w4, s2, b2);
-                    v[4 * m + 1] = dequant_pair<1>(w0, w4, s2, b2);
-                    v[4 * m + 2] = dequant_pair<2>(w0, w4, s2, b2);
-                    v[4 * m + 3] = dequant_pair<3>(w0, w4, s2, b2);
+                    // nibble pairs (j, j+4) of the word: the split order of every 8 inputs,
+                    // which the activation rows (xg, h) are stored in as well
+                    v[4 * m + 0] = dequant_split(w0, s2, b2);
+                    v[4 * m + 1] = dequant_split(w4, s2, b2);
+                    v[4 * m + 2] = dequant_split(w0 >> 8, s2, b2);
+                    v[4 * m + 3] = dequant_split(w0 >> 12, s2, b2);
                 }
             };
-            // two chunks per round: one tensor-memory store wait covers both
-            for (int kc = 0; kc < KC; kc += 2, it += 2) {
-                const int s0 = it % kStages, s1 = (it + 1) % kStages;
-                const uint32_t sb0 = sb_of(kc), sb1 = sb_of(kc + 1);
-                const uint32_t cit = it / cps;    // both chunks of the pair share a codes stage (cps even)
+            // one chunk per round: this warp's 64 inputs (one group) of 32 rows
+            for (int kc = 0; kc < KC; ++kc, ++it) {
+                const int s = it % kStages;
+                const int grp = 2 * kc + khalf;
+                const uint32_t sbw = sb_tma ? sbs_row[grp] : ldg_u32(sbrow + grp);
+                const uint32_t cit = it / cps;    // tiles hold whole codes stages
                 const int cs = cit % kCStages;
                 mbar_wait_bounded(&sm.cfull[cs], (cit / kCStages) & 1, a.err);
-                const uint4 cw0 = codes_at(cs, kc);
-                const uint4 cw1 = codes_at(cs, kc + 1);
-                if ((kc + 2) % cps == 0) {
+                const int u0 = (kc % cps) * 4 + khalf * 2;
+                const uint4 cw0 = codes_at(cs, u0);
+                const uint4 cw1 = codes_at(cs, u0 + 1);
+                if ((kc + 1) % cps == 0) {
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&sm.cempty[cs]);
                 }
                 uint32_t v0[16], v1[16];
-                dequant16(cw0, sb0, v0);
-                dequant16(cw1, sb1, v1);
-                // the MMA reads B from ring stage s0/s1: make sure it landed before
-                // the A operand of the same chunks is declared ready (the MMA
-                // also waits on it, this keeps the two rings in step)
-                if (it >= kStages) mbar_wait_bounded(&sm.mma_done[s0], ((it / kStages) - 1) & 1, a.err);
-                if (it + 1 >= kStages) mbar_wait_bounded(&sm.mma_done[s1], (((it + 1) / kStages) - 1) & 1, a.err);
+                dequant16(cw0, sbw, v0);
+                dequant16(cw1, sbw, v1);
+                // the tensor-memory A stage is free once the MMAs of its previous use completed
+                if (it >= kStages) mbar_wait_bounded(&sm.mma_done[s], ((it / kStages) - 1) & 1, a.err);
                 tc_fence_after();
-                tmem_st16(lane_addr + s0 * kAStageCols, v0);
-                tmem_st16(lane_addr + s1 * kAStageCols, v1);
+                tmem_st16(lane_addr + s * kAStageCols, v0);
+                tmem_st16(lane_addr + s * kAStageCols + 16, v1);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&sm.a_full[s0]);
-                    mbar_arrive(&sm.a_full[s1]);
-                }
+                if (lane == 0) mbar_arrive(&sm.a_full[s]);
             }
             if (sb_tma) {
                 __syncwarp();
@@ -442,7 +439,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int col = c0 + c + odd;
                         if (col < tl.nr) {
                             const float hval = __fdividef(gate, 1.0f + __expf(-gate)) * up;
-                            a.h[(tl.hrow0 + col) * a.I + j] = f32_to_bf16(hval);
+                            // h is kept in the split order inside every 8 columns (the down
+                            // GEMM's dequantised weights come in that order)
+                            const int js = (j & ~7) | ((j & 4) ? 2 * (j & 3) + 1 : 2 * (j & 3));
+                            a.h[(tl.hrow0 + col) * a.I + js] = f32_to_bf16(hval);
                         }
                     }
                 } else {
@@ -511,16 +511,17 @@ bool make_codes_map(CUtensorMap* m, const uint32_t* codes, int rows, int K, int 
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// bf16 [rows, cols] activations read in boxes of 64 columns (128 bytes) x
-// box_rows rows, 128B-swizzled (the K-major layout the MMA reads).
+// bf16 [rows, cols] activations as a 3-D view (64 columns of a 64-column
+// block, row, block), read in boxes of box_rows rows x two blocks (128
+// columns), each block 128B-swizzled: the K-major layout the MMA reads.
 bool make_act_map(CUtensorMap* m, const uint16_t* base, int rows, int cols, int box_rows) {
     EncodeTiled enc = encode_fn();
     if (!enc) return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(base), dims, strides, box, estr,
+    const cuuint64_t dims[3] = {64, (cuuint64_t)rows, (cuuint64_t)(cols / 64)};
+    const cuuint64_t strides[2] = {(cuuint64_t)cols * 2, 128};
+    const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -549,7 +550,8 @@ int num_sms() {
 }
 
 // xg[r] = x[token of row r]: routed rows in expert order (row_to_pair), then
-// the shared expert's rows (tokens 0..T-1).  One warp per row, 16-byte moves.
+// the shared expert's rows (tokens 0..T-1), each 8 inputs in the split order.
+// One warp per row, 16-byte moves.
 __global__ void __launch_bounds__(256) k_gather_rows(FfnArgs a) {
     const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
     const int rows = (a.K + 1) * a.T;
@@ -564,25 +566,38 @@ __global__ void __launch_bounds__(256) k_gather_rows(FfnArgs a) {
     }
     const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)tok * a.H);
     uint4* dst = reinterpret_cast<uint4*>(a.xg + (size_t)row * a.H);
-    for (int c = lane; c < a.H / 8; c += 32) dst[c] = src[c];
+    // each 8 inputs in the split order (0,4,1,5,2,6,3,7) of the dequantised weights
+    for (int c = lane; c < a.H / 8; c += 32) {
+        const uint4 v = src[c];
+        uint4 r;
+        r.x = prmt(v.x, v.z, 0x5410);
+        r.y = prmt(v.x, v.z, 0x7632);
+        r.z = prmt(v.y, v.w, 0x5410);
+        r.w = prmt(v.y, v.w, 0x7632);
+        dst[c] = r;
+    }
 }
 
 }  // namespace
 
 bool ffn_tc_supported(const FfnArgs& a) {
-    // chunks are taken two at a time: K/64 even for both GEMMs
-    // one tile's (scale, bias) rows must fit their shared-memory buffer
-    return a.E <= 256 && a.K == 8 && a.G == 64 && a.H % 128 == 0 && a.I % 128 == 0 && a.H >= 128 && a.I >= 128 &&
-           128 * (a.H / 64) * 4 <= kSbBytes && 128 * (a.I / 64) * 4 <= kSbBytes;
+    // a codes stage (256 inputs, or all of K when K is 128) holds whole chunks
+    // of 128 inputs and every tile whole stages: K is 128 or a multiple of 256
+    // for both GEMMs; one tile's (scale, bias) rows must fit their buffer
+    auto k_ok = [](int k) { return k == 128 || (k >= 256 && k % 256 == 0); };
+    return a.E <= 256 && a.K == 8 && a.G == 64 && k_ok(a.H) && k_ok(a.I) && 128 * (a.H / 64) * 4 <= kSbBytes &&
+           128 * (a.I / 64) * 4 <= kSbBytes;
 }
 
 cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     const int nmat = a.E + 1;
-    CUtensorMap gu_map, d_map, x_map, h_map;
+    CUtensorMap gu_map, d_map, x_map, h_map, x_map128, h_map128;
     if (!make_codes_map(&gu_map, a.gu_codes, nmat * 2 * a.I, a.H, 64)) return cudaErrorInvalidValue;
     if (!make_codes_map(&d_map, a.d_codes, nmat * a.H, a.I, 128)) return cudaErrorInvalidValue;
     if (!make_act_map(&x_map, a.xg, (a.K + 1) * a.T, a.H, 64)) return cudaErrorInvalidValue;
     if (!make_act_map(&h_map, a.h, (a.K + 1) * a.T, a.I, 64)) return cudaErrorInvalidValue;
+    if (!make_act_map(&x_map128, a.xg, (a.K + 1) * a.T, a.H, 128)) return cudaErrorInvalidValue;
+    if (!make_act_map(&h_map128, a.h, (a.K + 1) * a.T, a.I, 128)) return cudaErrorInvalidValue;
     // (scale, bias) maps only when a row's words fill whole 16-byte units
     CUtensorMap gsb_map = gu_map, dsb_map = d_map;
     if ((a.H / 64) % 4 == 0 && !make_sb_map(&gsb_map, a.gu_sb, nmat * 2 * a.I, a.H, 64)) return cudaErrorInvalidValue;
@@ -598,11 +613,11 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     TcArgs ta;
     ta.f = a;
     ta.gateup = 1;
-    k_ffn_tc<<<G, kThreads, smem, st>>>(gu_map, x_map, gsb_map, ta);
+    k_ffn_tc<<<G, kThreads, smem, st>>>(gu_map, x_map, x_map128, gsb_map, ta);
     ce = cudaGetLastError();
     if (ce != cudaSuccess) return ce;
     ta.gateup = 0;
-    k_ffn_tc<<<G, kThreads, smem, st>>>(d_map, h_map, dsb_map, ta);
+    k_ffn_tc<<<G, kThreads, smem, st>>>(d_map, h_map, h_map128, dsb_map, ta);
     return cudaGetLastError();
 }
 

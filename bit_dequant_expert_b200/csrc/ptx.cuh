@@ -338,7 +338,14 @@ __device__ __forceinline__ void tma_gather4(void* dst_smem, const void* tmap, in
         : "memory");
 }
 
-// Tiled loads of 4-D and 5-D boxes (no multicast); coordinates innermost first.
+// Tiled loads of 3-D, 4-D and 5-D boxes (no multicast); coordinates innermost first.
+__device__ __forceinline__ void tma_load_3d(void* dst_smem, const void* tmap, int c0, int c1, int c2, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+            smem_u32(dst_smem)),
+        "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+        : "memory");
+}
 __device__ __forceinline__ void tma_load_4d(void* dst_smem, const void* tmap, int c0, int c1, int c2, int c3,
                                             uint64_t* bar) {
     asm volatile(
