@@ -359,7 +359,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t* sbrow = sbase + (size_t)wrow * ngroups;
             const int buf = lt & 1;
             // this row's (scale, bias) words in shared memory: gate rows 0..63, up rows 64..127
-            const uint32_t* sbs_row = sm.sbs[buf] + (size_t)(gateup ? ((L & 1) * 64 + (L >> 1)) : L) * ngroups;
+            const int srow = gateup ? ((L & 1) * 64 + (L >> 1)) : L;
+            const uint32_t* sbs_row = sm.sbs[buf] + (size_t)srow * ngroups;
             if (sb_tma) mbar_wait_bounded(&sm.sb_full[buf], (lt >> 1) & 1, a.err);
             auto dequant16 = [&](uint4 cw, uint32_t sbw, uint32_t* v) {
                 const uint32_t s2 = prmt(sbw, sbw, 0x1010), b2 = prmt(sbw, sbw, 0x3232);
@@ -379,7 +380,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kc = 0; kc < KC; ++kc, ++it) {
                 const int s = it % kStages;
                 const int grp = 2 * kc + khalf;
-                const uint32_t sbw = sb_tma ? sbs_row[grp] : ldg_u32(sbrow + grp);
+                // 128-byte (scale, bias) rows are 128B-swizzled: word g of row r at unit (g/4) ^ (r&7)
+                const uint32_t sbw = !sb_tma ? ldg_u32(sbrow + grp)
+                                     : ngroups == 32 ? sbs_row[(((grp >> 2) ^ (srow & 7)) << 2) | (grp & 3)]
+                                                     : sbs_row[grp];
                 const uint32_t cit = it / cps;    // tiles hold whole codes stages
                 const int cs = cit % kCStages;
                 mbar_wait_bounded(&sm.cfull[cs], (cit / kCStages) & 1, a.err);
@@ -445,20 +449,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                             a.h[(tl.hrow0 + col) * a.I + js] = f32_to_bf16(hval);
                         }
                     }
+                } else if (a.mode != MOE_MODE_SCATTER) {
+                    // bf16 rows: lanes 2i / 2i+1 swap one column so that each writes two
+                    // adjacent outputs (n, n+1) of one token row with a 32-bit store
+                    const int n = 128 * tl.mb + 32 * q + lane;
+                    const int odd = lane & 1;
+                    uint16_t* dst = tl.e == a.E ? a.y_shared : a.y_rows;
+#pragma unroll
+                    for (int c = 0; c < 16; c += 2) {
+                        const float y0 = __uint_as_float(v[c]), y1 = __uint_as_float(v[c + 1]);
+                        const float recv = __shfl_xor_sync(0xFFFFFFFFu, odd ? y0 : y1, 1);
+                        const int col = c0 + c + odd;
+                        const uint32_t pk = odd ? pack_bf16x2(recv, y1) : pack_bf16x2(y0, recv);
+                        if (col < tl.nr)
+                            *reinterpret_cast<uint32_t*>(dst + (size_t)(tl.r0 + col) * a.H + (n & ~1)) = pk;
+                    }
                 } else {
+                    // fp32 y_acc: w * y added into the token's row
                     const int n = 128 * tl.mb + 32 * q + lane;
 #pragma unroll
                     for (int c = 0; c < 16; ++c) {
                         const int col = c0 + c;
-                        if (col >= tl.nr) break;
-                        const float y = __uint_as_float(v[c]);
-                        if (a.mode == MOE_MODE_SCATTER) {
-                            atomicAdd(a.y_acc + (size_t)sm.tok[slot][col] * a.H + n, sm.w[slot][col] * y);
-                        } else if (tl.e == a.E) {
-                            a.y_shared[(size_t)(tl.r0 + col) * a.H + n] = f32_to_bf16(y);
-                        } else {
-                            a.y_rows[(size_t)(tl.r0 + col) * a.H + n] = f32_to_bf16(y);
-                        }
+                        if (col < tl.nr)
+                            atomicAdd(a.y_acc + (size_t)sm.tok[slot][col] * a.H + n,
+                                      sm.w[slot][col] * __uint_as_float(v[c]));
                     }
                 }
             }
@@ -536,9 +550,11 @@ bool make_sb_map(CUtensorMap* m, const uint16_t* sb, int rows, int K, int box_ro
     const cuuint64_t strides[1] = {(cuuint64_t)ng * 4};
     const cuuint32_t box[2] = {(cuuint32_t)ng, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
+    // 128-byte rows land 128B-swizzled, so the 32 rows one load instruction
+    // touches spread over the banks
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint16_t*>(sb), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+               CU_TENSOR_MAP_INTERLEAVE_NONE, ng == 32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 int num_sms() {
