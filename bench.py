@@ -119,6 +119,42 @@ class ClockSampler:
 # ------------------------------------------------------------ distributed
 
 
+# Kernel sources whose ncu summaries under profiles/ carry DRAM traffic per launch.
+KERNEL_SOURCES = {
+    "ffn_gemv": ["bit_dequant_expert_b200/csrc/ffn_gemv.cu"],
+    "ffn_tc": ["bit_dequant_expert_b200/csrc/ffn_tc.cu"],
+}
+KERNEL_HEADERS = ["bit_dequant_expert_b200/csrc/common.cuh", "bit_dequant_expert_b200/csrc/ptx.cuh",
+                  "bit_dequant_expert_b200/csrc/topk.cuh", "bit_dequant_expert_b200/csrc/kernels.h"]
+
+
+def kernel_source_hash(name: str) -> str:
+    """sha256 over a kernel's source file and the headers it includes."""
+    import hashlib
+    h = hashlib.sha256()
+    root = os.path.dirname(os.path.abspath(__file__))
+    for rel in KERNEL_SOURCES[name] + KERNEL_HEADERS:
+        with open(os.path.join(root, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(name: str, summary: str):
+    """DRAM bytes (read + write) per launch from profiles/<summary>, or None when
+    the summary is missing or the kernel's sources changed since it was taken."""
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles", summary)
+    try:
+        fields = dict(line.split(":", 1) for line in open(path).read().splitlines() if ":" in line)
+    except OSError:
+        return None
+    if fields.get("source_sha256", "").strip() != kernel_source_hash(name):
+        return None
+    try:
+        return int(fields["traffic_bytes_per_launch"].strip())
+    except (KeyError, ValueError):
+        return None
+
+
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -266,7 +302,8 @@ def run_decode(device, steps, warmup, world, peaks):
         ffn_ms = _timed_replays(g_ffn.replay, steps, stream) / (steps * LAYERS)
     achieved = FFN_BYTES_T1 / (ffn_ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "frac": achieved / peaks["hbm_gbs"],
+                "traffic": profiled_traffic("ffn_gemv", "ffn_gemv_decode_t1_ncu.txt"),
                 "kernel": "moe_expert_ffn (T=1: gate/up + SwiGLU, then down + combine-add)",
                 "algorithmic_bytes": FFN_BYTES_T1, "avg_launch_us": ffn_ms * 1e3,
                 "peak_source": peaks["source"] + " hbm_gbs"}
@@ -358,7 +395,8 @@ def run_prefill(device, steps, warmup, world, peaks):
             "value": T / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms, "steps": steps,
             "ffn_ms": ffn_ms,
             "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": tflops / peaks["bf16_tflops"], "traffic": None,
+                         "frac": tflops / peaks["bf16_tflops"],
+                         "traffic": profiled_traffic("ffn_tc", "ffn_tc_prefill_t2048_ncu.txt"),
                          "kernel": "moe_expert_ffn (T=2048)", "algorithmic_flops": flops,
                          "peak_source": peaks["source"] + " bf16_tflops (burst)",
                          "hbm_frac_of_weight_bytes": wbytes / (ffn_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
