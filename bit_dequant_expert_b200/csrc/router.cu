@@ -238,9 +238,12 @@ cudaError_t launch_router(const RouterArgs& a, cudaStream_t st) {
     const float* lg = a.logits_in;
     const float* topk_bias = a.bias;
     if (!lg) {
-        dim3 grid((a.T + 7) / 8, a.E / 64);
-        k_router_logits<8, 8><<<grid, 256, 0, st>>>(a.T, a.H, a.E, a.x, a.w_router, a.bias, a.bias_stride,
-                                                     a.logits_ws, a.counts);
+        // 4 tokens x 16 experts per warp, 8 warps over 128 experts: the x chunk of
+        // a token is widened once for 16 experts, and the small accumulator tile
+        // leaves room for two blocks per SM
+        dim3 grid((a.T + 3) / 4, a.E / 128);
+        k_router_logits<4, 16><<<grid, 256, 0, st>>>(a.T, a.H, a.E, a.x, a.w_router, a.bias, a.bias_stride,
+                                                      a.logits_ws, a.counts);
         lg = a.logits_ws;
         topk_bias = nullptr;
     } else {
