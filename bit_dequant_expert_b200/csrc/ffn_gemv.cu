@@ -301,12 +301,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
 #pragma unroll
                 for (int t = 0; t < kMaxT; ++t) {
-                    float v = acc[t];
+                    if (t < T) {   // T is the same for the whole warp
+                        float v = acc[t];
 #pragma unroll
-                    for (int off = 16; off >= 1; off >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xFFFFFFFFu, v, off));
-                    if (lane == t && t < T) {
-                        if (ga.r.bias) v = __fadd_rn(v, ga.r.bias[(int64_t)t * ga.r.bias_stride + r_e]);
-                        ga.r.logits[(size_t)t * E + r_e] = v;
+                        for (int off = 16; off >= 1; off >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xFFFFFFFFu, v, off));
+                        if (lane == t) {
+                            if (ga.r.bias) v = __fadd_rn(v, ga.r.bias[(int64_t)t * ga.r.bias_stride + r_e]);
+                            ga.r.logits[(size_t)t * E + r_e] = v;
+                        }
                     }
                 }
             }

@@ -195,12 +195,14 @@ __global__ void __launch_bounds__(64) k_route_small_wide(int T, int H, int E, co
     }
 #pragma unroll
     for (int t = 0; t < 8; ++t) {
-        float v = acc[t];
+        if (t < T) {   // T is the same for the whole warp
+            float v = acc[t];
 #pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xFFFFFFFFu, v, off));
-        if (lane == t && t < T) {
-            if (bias) v = __fadd_rn(v, bias[(int64_t)t * bias_stride + e]);
-            logits[(size_t)t * E + e] = v;
+            for (int off = 16; off >= 1; off >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xFFFFFFFFu, v, off));
+            if (lane == t) {
+                if (bias) v = __fadd_rn(v, bias[(int64_t)t * bias_stride + e]);
+                logits[(size_t)t * E + e] = v;
+            }
         }
     }
     __threadfence();
