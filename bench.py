@@ -129,13 +129,18 @@ KERNEL_HEADERS = ["bit_dequant_expert_b200/csrc/common.cuh", "bit_dequant_expert
 
 
 def kernel_source_hash(name: str) -> str:
-    """sha256 over a kernel's source file and the headers it includes."""
+    """sha256 over the code of a kernel's source file and the headers it
+    includes: `//` comments, trailing blanks and empty lines do not count."""
     import hashlib
+    import re
     h = hashlib.sha256()
     root = os.path.dirname(os.path.abspath(__file__))
     for rel in KERNEL_SOURCES[name] + KERNEL_HEADERS:
-        with open(os.path.join(root, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(root, rel)) as f:
+            for line in f:
+                code = re.sub(r"(^|\s)//.*$", "", line).rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()
 
 

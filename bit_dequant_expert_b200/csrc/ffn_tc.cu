@@ -8,25 +8,26 @@
 // paragraph (folding the dequantisation into the matrix multiplication so an
 // expanded array never touches memory: +77.4% prefill at 512 tokens).
 //
-// One persistent kernel template, instantiated for gate/up (+SwiGLU) and for
+// One persistent kernel, launched once for gate/up (+SwiGLU) and once for
 // down (+weighted combine).  A tile is 128 weight rows (MMA M) x up to 128
-// token rows (MMA N) of one expert; K runs in 64-input chunks, one (scale,
-// bias) group each.  Per chunk:
-//   warp 0       TMA: the tile's 128 rows x 64 codes (4 KB) and the B operand
-//                rows (x rows already gathered into expert order for gate/up,
-//                h rows for down; contiguous either way) into one smem ring
-//                stage; B lands 128B-swizzled and K-major, as the MMA reads it;
-//   warps 2-3    TMA of the B boxes (alternate chunks: one thread keeps only
-//                one box in flight at a time) and, for down, each tile's
-//                per-column token and routing weight for the epilogue;
-//   warps 4-11   dequantise codes to bf16 (scale * q + bias) and write them as
-//                the A operand straight into tensor memory (tcgen05.st), so
-//                the MMA reads only B from shared memory;
-//   warp 1       one thread issues 4 tcgen05.mma (K = 16 each) into one of two
-//                TMEM accumulators and commits to mbarriers;
+// token rows (MMA N) of one expert; K runs in 128-input stages (two (scale,
+// bias) groups), three stages in flight.  Roles:
+//   warp 0       TMA of the codes (128 rows x 256 inputs per 16 KB box, two
+//                stages, 128B-swizzled) and of each tile's (scale, bias) rows;
+//   warps 2-3    one 3-D TMA box per stage of the B operand: the tile's token
+//                rows (x gathered into expert order for gate/up, h for down),
+//                two 64-input halves, 128B-swizzled and K-major as the MMA
+//                reads them; alternate stages each; for down also each
+//                tile's per-column token and routing weight;
+//   warps 4-11   dequantise codes to bf16 (scale * q + bias; a code word
+//                gives the nibble pairs (j, j+4), and x and h are stored in
+//                that order inside every 8 inputs) and write them as the A
+//                operand straight into tensor memory (tcgen05.st);
+//   warp 1       one thread issues 8 tcgen05.mma (K = 16 each) per stage into
+//                one of two TMEM accumulators and commits to mbarriers;
 //   warps 12-15  epilogue from TMEM: SwiGLU (gate and up rows interleaved on
-//                adjacent TMEM lanes) -> h in bf16, or w * y scattered into
-//                y_acc (fp32 red) / bf16 rows.
+//                adjacent TMEM lanes) -> h in bf16, or bf16 rows (paired
+//                32-bit stores) / w * y added into y_acc (fp32 red).
 // Every wait is bounded (error word MOE_ERR_TIMEOUT, never a hang).
 #include <cuda.h>
 
