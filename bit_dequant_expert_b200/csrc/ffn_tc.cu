@@ -169,9 +169,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int KC = K / kBK;                      // chunks per tile
     const int ngroups = K / 64;
     // codes come in stages of cw u32 words (8 cw inputs) per row: 256 inputs,
-    // or all of K when K is shorter; a stage feeds cps chunks
+    // or all of K when K is shorter; a stage feeds 1 << cps_sh chunks
     const int cw = K >= 256 ? 32 : K / 8;
-    const int cps = cw / 16;
+    const int cps_sh = cw == 32 ? 1 : 0;         // a stage feeds 1 << cps_sh chunks
+    const int cps_mask = (1 << cps_sh) - 1;
     // (scale, bias) rows go through shared memory by TMA when a row's words
     // span whole 16-byte units; otherwise (tiny K) each thread reads its own
     const bool sb_tma = (ngroups & 3) == 0;
@@ -220,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
-        // (scale, bias) rows once per tile, codes once per stage of cps chunks;
+        // (scale, bias) rows once per tile, codes once per stage of 1 << cps_sh chunks;
         // a stage is refilled once its chunks were dequantised.
         uint32_t it = 0, lt = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
@@ -238,9 +239,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             for (int kc = 0; kc < KC; ++kc, ++it) {
                 if (lane == 0) {
-                    if (kc % cps == 0) {
-                        const uint32_t cit = it / cps;        // tiles hold whole codes stages
-                        const int cs = cit % kCStages;
+                    if ((kc & cps_mask) == 0) {
+                        const uint32_t cit = it >> cps_sh;    // tiles hold whole codes stages
+                        const int cs = cit & (kCStages - 1);
                         if (cit >= kCStages) mbar_wait_bounded(&sm.cempty[cs], ((cit / kCStages) - 1) & 1, a.err);
                         mbar_arrive_expect_tx(&sm.cfull[cs], 128 * cw * 4);
                         if (gateup) {
@@ -257,7 +258,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            uint32_t it = 0, lt = 0;
+            uint32_t lt = 0, par = 0;
+            int s = 0;   // ring stage and its phase, advanced per chunk
             for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
                 const Tile tl = decode_tile(a, gateup, sm.pre, sm.off, t);
                 const int ab = lt & 1;
@@ -265,9 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint32_t idesc = idesc_bf16_f32(128, tl.npad);
                 const uint32_t d_tmem = tmem + ab * kNT;
-                for (int kc = 0; kc < KC; ++kc, ++it) {
-                    const int s = it % kStages;
-                    const uint32_t par = (it / kStages) & 1;
+                for (int kc = 0; kc < KC; ++kc) {
                     mbar_wait_bounded(&sm.a_full[s], par, a.err);
                     mbar_wait_bounded(&sm.full[s], par, a.err);
                     tc_fence_after();
@@ -281,6 +281,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc_mma_ts(d_tmem, a_tmem + 8 * j, (j < 4 ? bdesc0 : bdesc1) + 2 * (j & 3), idesc,
                                   (kc | j) != 0);
                     tc_commit(&sm.mma_done[s]);
+                    if (++s == kStages) {
+                        s = 0;
+                        par ^= 1u;
+                    }
                 }
                 tc_commit(&sm.acc_full[ab]);
             }
@@ -291,7 +295,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // B boxes are issued by two warps, alternate chunks each.
         const int bt = tid - 64;
         const uint32_t par = warp - 2;
-        uint32_t it = 0, lt = 0;
+        uint32_t it = 0, lt = 0, bph = 0;
+        int bst = 0;   // ring stage of chunk it and its phase
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
             const Tile tl = decode_tile(a, gateup, sm.pre, sm.off, t);
             if (!gateup) {
@@ -325,10 +330,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             // one 3-D box per chunk: R token rows x two 64-input halves
             const int R = tl.npad > 64 ? 128 : 64;
             for (int kc = 0; kc < KC; ++kc, ++it) {
+                const int s = bst;
+                const uint32_t ph = bph;
+                if (++bst == kStages) {
+                    bst = 0;
+                    bph ^= 1u;
+                }
                 if ((it & 1u) != par) continue;
-                const int s = it % kStages;
                 if (lane == 0) {
-                    if (it >= kStages) mbar_wait_bounded(&sm.mma_done[s], ((it / kStages) - 1) & 1, a.err);
+                    if (it >= kStages) mbar_wait_bounded(&sm.mma_done[s], ph ^ 1u, a.err);
                     mbar_arrive_expect_tx(&sm.full[s], R * 2 * 128);
                     tma_load_3d(sm.b[s], R == 128 ? &b_map128 : &b_map64, 0, (int)tl.hrow0, 2 * kc, &sm.full[s]);
                 }
@@ -353,7 +363,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int phys = cw == 32 ? (u ^ (crow & 7)) : u;
             return *reinterpret_cast<const uint4*>(sm.codes[cs] + crow * cw * 4 + phys * 16);
         };
-        uint32_t it = 0, lt = 0;
+        uint32_t it = 0, lt = 0, dph = 0;
+        int dst = 0;   // ring stage of chunk it and its phase
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
             const Tile tl = decode_tile(a, gateup, sm.pre, sm.off, t);
             const int wrow = gateup ? ((L & 1) ? wrow_up(a, tl) : wrow_gate(a, tl)) + (L >> 1) : wrow_down(a, tl) + L;
@@ -379,19 +390,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             // one chunk per round: this warp's 64 inputs (one group) of 32 rows
             for (int kc = 0; kc < KC; ++kc, ++it) {
-                const int s = it % kStages;
+                const int s = dst;
+                const uint32_t ph = dph;
+                if (++dst == kStages) {
+                    dst = 0;
+                    dph ^= 1u;
+                }
                 const int grp = 2 * kc + khalf;
                 // 128-byte (scale, bias) rows are 128B-swizzled: word g of row r at unit (g/4) ^ (r&7)
                 const uint32_t sbw = !sb_tma ? ldg_u32(sbrow + grp)
                                      : ngroups == 32 ? sbs_row[(((grp >> 2) ^ (srow & 7)) << 2) | (grp & 3)]
                                                      : sbs_row[grp];
-                const uint32_t cit = it / cps;    // tiles hold whole codes stages
-                const int cs = cit % kCStages;
+                const uint32_t cit = it >> cps_sh;    // tiles hold whole codes stages
+                const int cs = cit & (kCStages - 1);
                 mbar_wait_bounded(&sm.cfull[cs], (cit / kCStages) & 1, a.err);
-                const int u0 = (kc % cps) * 4 + khalf * 2;
+                const int u0 = (kc & cps_mask) * 4 + khalf * 2;
                 const uint4 cw0 = codes_at(cs, u0);
                 const uint4 cw1 = codes_at(cs, u0 + 1);
-                if ((kc + 1) % cps == 0) {
+                if (((kc + 1) & cps_mask) == 0) {
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&sm.cempty[cs]);
                 }
@@ -399,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 dequant16(cw0, sbw, v0);
                 dequant16(cw1, sbw, v1);
                 // the tensor-memory A stage is free once the MMAs of its previous use completed
-                if (it >= kStages) mbar_wait_bounded(&sm.mma_done[s], ((it / kStages) - 1) & 1, a.err);
+                if (it >= kStages) mbar_wait_bounded(&sm.mma_done[s], ph ^ 1u, a.err);
                 tc_fence_after();
                 tmem_st16(lane_addr + s * kAStageCols, v0);
                 tmem_st16(lane_addr + s * kAStageCols + 16, v1);
