@@ -1,5 +1,7 @@
-// Thin inline-PTX wrappers (sm_100a): mbarriers with bounded waits, bulk
-// async copies, named barriers, legacy warp MMA, and a global timer.
+// Thin inline-PTX wrappers (sm_100a): mbarriers with bounded waits, TMA tiled
+// loads, named barriers, dependent-launch control, warp MMA, tensor-memory
+// allocation / loads / stores and tcgen05.mma, 4-bit dequantisation, vector
+// reductions and a global timer.
 #pragma once
 
 #include <stdint.h>
@@ -79,15 +81,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
 
 // ------------------------------------------------------------------ copies
 
-// 1-D bulk async copy global -> shared, completion counted in bytes on `bar`.
-// Both addresses 16-byte aligned, bytes a multiple of 16.
-__device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, uint32_t bytes, uint64_t* bar) {
-    asm volatile("cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     smem_u32(dst_smem)),
-                 "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar))
-                 : "memory");
-}
-
 // ------------------------------------------------------------------ sync
 
 __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t nthreads) {
@@ -99,70 +92,7 @@ __device__ __forceinline__ void named_barrier_arrive(uint32_t id, uint32_t nthre
     asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// ------------------------------------------------------------------ clusters and dependent launches
-
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-// Every thread of every CTA of the cluster arrives, then waits for the rest.
-__device__ __forceinline__ void cluster_sync_all() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// Address of the same shared-memory location in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-    return r;
-}
-
-__device__ __forceinline__ void st_cluster_u16(uint32_t caddr, uint16_t v) {
-    asm volatile("st.shared::cluster.u16 [%0], %1;" ::"r"(caddr), "h"(v) : "memory");
-}
-
-__device__ __forceinline__ void st_cluster_u32(uint32_t caddr, uint32_t v) {
-    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(caddr), "r"(v) : "memory");
-}
-
-// Arrive (release, cluster scope) on an mbarrier given by its shared::cluster
-// address, which may live in another CTA of the cluster.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t caddr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
-}
-
-// Bounded wait with cluster-scope acquire: what other CTAs of the cluster
-// wrote before their release-arrive is visible afterwards.
-__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_t parity, int32_t* err,
-                                                          uint64_t limit_ns = 200000000ull) {
-    auto try_once = [&]() {
-        uint32_t ok;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(ok)
-            : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
-            : "memory");
-        return ok != 0;
-    };
-    if (try_once()) return true;
-    const uint64_t t0 = globaltimer_ns();
-    while (!try_once()) {
-        if (globaltimer_ns() - t0 > limit_ns) {
-            if (err) atomicCAS(err, 0, 6 /* MOE_ERR_TIMEOUT */);
-            return false;
-        }
-    }
-    return true;
-}
+// ------------------------------------------------------------------ dependent launches
 
 // Programmatic dependent launch: wait for the grid this one depends on (a
 // no-op when launched without the attribute), and let the next grid on the
@@ -173,12 +103,6 @@ __device__ __forceinline__ void griddep_launch_dependents() {
 }
 
 // ------------------------------------------------------------------ mma
-
-__device__ __forceinline__ void ldmatrix_x4(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3, const void* p) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(smem_u32(p)));
-}
 
 // D += A(16x16 bf16, row) * B(16x8 bf16, col), fp32 accumulate.
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -205,15 +129,6 @@ __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint3
     return d;
 }
 
-// bf16x2 (128 + q[2p], 128 + q[2p+1]) from nibbles 2p, 2p+1 of word v
-// (v4 = v >> 4).  0x43 is the high byte of bf16 128; the nibble fills the
-// low mantissa bits, so the value is exact.
-template <int P>
-__device__ __forceinline__ uint32_t nibble_pair_biased(uint32_t v, uint32_t v4) {
-    constexpr uint32_t sel = P | (P << 4) | ((4 + P) << 8) | ((4 + P) << 12);
-    return lop3_and_or(prmt(v, v4, sel), 0x000F000Fu, 0x43004300u);
-}
-
 __device__ __forceinline__ uint32_t hsub2_bf16(uint32_t a, uint32_t b) {
     uint32_t d;
     asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
@@ -234,15 +149,6 @@ __device__ __forceinline__ uint32_t nibble_pair_split(uint32_t vs) { return lop3
 // j+4 of a code word; vs is the word shifted right by 4j.
 __device__ __forceinline__ uint32_t dequant_split(uint32_t vs, uint32_t s2, uint32_t b2) {
     return hfma2_bf16(hsub2_bf16(nibble_pair_split(vs), 0x43004300u), s2, b2);
-}
-
-// Dequantised bf16x2 weights of nibbles 2p, 2p+1: scale * q + bias, rounded
-// once (the product scale * q is exact inside the fma).  s2 / b2 hold the
-// bf16 scale / bias in both halves.
-template <int P>
-__device__ __forceinline__ uint32_t dequant_pair(uint32_t v, uint32_t v4, uint32_t s2, uint32_t b2) {
-    const uint32_t q = hsub2_bf16(nibble_pair_biased<P>(v, v4), 0x43004300u);
-    return hfma2_bf16(q, s2, b2);
 }
 
 // ------------------------------------------------------------------ tensor memory (tcgen05)
@@ -300,19 +206,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// 32 consecutive 32-bit columns of this thread's lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
-        "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
-          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
-          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-        : "r"(taddr)
-        : "memory");
-}
-
 // Shared-memory matrix descriptor: K-major operand in the canonical
 // 128-byte-swizzled layout (8-row groups of 128-byte rows, 1024 bytes apart).
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
@@ -337,17 +230,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst_smem, const void* tmap, in
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
             smem_u32(dst_smem)),
         "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar))
-        : "memory");
-}
-
-// Four rows (row0..row3) x one box width of a 2-D tensor whose box is one
-// row high, written as four consecutive box rows at dst.
-__device__ __forceinline__ void tma_gather4(void* dst_smem, const void* tmap, int x, int r0, int r1, int r2, int r3,
-                                            uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
-        "%4, %5, %6}], [%7];" ::"r"(smem_u32(dst_smem)),
-        "l"(tmap), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
         : "memory");
 }
 
@@ -387,15 +269,6 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
                  : "memory");
 }
 
-// Starts pulling `bytes` (a multiple of 16, 16-byte aligned) into L2.
-__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-
-// 16-byte async copy global -> shared; src_bytes 0 fills zeros.
-__device__ __forceinline__ void cp_async16(uint32_t dst_saddr, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst_saddr), "l"(src), "r"(src_bytes) : "memory");
-}
 // 4-byte async copy global -> shared (both 4-byte aligned).
 __device__ __forceinline__ void cp_async4(uint32_t dst_saddr, const void* src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst_saddr), "l"(src) : "memory");
@@ -404,9 +277,6 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 }  // namespace moe
