@@ -101,3 +101,20 @@ def test_decode_layer_validation_before_launch():
     assert _decode(cfg, 8, need, x=None) == m.MOE_ERR_INVALID_ARG
     assert _decode(cfg, 8, need, y=FAKE + 8) == m.MOE_ERR_INVALID_ARG
     assert _decode(cfg, 8, need, bias=FAKE, stride=-1) == m.MOE_ERR_INVALID_ARG
+
+
+def test_launch_count_per_path():
+    """Kernels per layer as the bench counts them (host-only, no device needed)."""
+    import bit_dequant_expert_b200 as m
+    cfg = m.config()
+    SC, PA = m.MOE_MODE_SCATTER, m.MOE_MODE_PAIRS
+    # route (small T: one launch) + permute (T <= 256: one) + decode FFN (one) + combine
+    assert m.moe_launch_count(cfg, 1, SC, m.MOE_PATH_AUTO) == 4
+    # the decode kernel only accumulates y_acc: bf16 rows go to the tensor-core path (gather + 2)
+    assert m.moe_launch_count(cfg, 1, PA, m.MOE_PATH_AUTO) == 1 + 1 + 3 + 1
+    # T = 2048: router logits + top-k, three permute kernels, gather + two GEMMs, combine
+    assert m.moe_launch_count(cfg, 2048, PA, m.MOE_PATH_AUTO) == 2 + 3 + 3 + 1
+    assert m.moe_launch_count(cfg, 2048, SC, m.MOE_PATH_SIMT) == 2 + 3 + 2 + 1
+    assert m.moe_launch_count(cfg, 2048, SC, m.MOE_PATH_GEMV) == -1      # more than 8 tokens
+    assert m.moe_launch_count(cfg, 4, 7, m.MOE_PATH_AUTO) == -1          # no such mode
+    assert m.moe_launch_count(cfg, 0, SC, m.MOE_PATH_AUTO) == -1
