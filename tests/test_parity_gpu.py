@@ -408,3 +408,48 @@ def test_tc_and_simt_against_oracle(T):
     tok = _sample_tokens(T, 12, T + 5)
     check_output(dict(y=yt), lay, tok)
     check_output(dict(y=ys), lay, tok)
+
+
+@pytest.mark.parametrize("T", [1, 5])
+def test_fused_decode_layer_chain_in_graph(T):
+    """Three layers chained as in a decode step (each layer's input is the
+    previous layer's output), captured in one CUDA graph so the kernels run
+    with programmatic dependent launch: every layer must see its input only
+    after the previous layer finished writing it."""
+    import torch
+    import bit_dequant_expert_b200 as m
+    from bit_dequant_expert_b200.layer import MoELayer, to_device
+    spec = gen.config(0).with_T(T)
+    lays = [gen.make_layer(spec, l) for l in range(3)]
+    Ls = [MoELayer(lay, max_tokens=T) for lay in lays]
+    assert all(L.fused_ok(T) for L in Ls)
+    x0 = to_device(lays[0]["x"], "cuda")
+    ys = [torch.empty(T, Ls[0].H, dtype=torch.bfloat16, device="cuda") for _ in lays]
+
+    def chain():
+        inp = x0
+        for L, y in zip(Ls, ys):
+            L.forward(inp, y_out=y)
+            inp = y
+
+    st = torch.cuda.Stream()
+    with torch.cuda.stream(st):
+        chain()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=st):
+        chain()
+    for y in ys:
+        y.zero_()
+    with torch.cuda.stream(st):
+        for _ in range(3):
+            g.replay()
+    torch.cuda.synchronize()
+    for l, (L, lay) in enumerate(zip(Ls, lays)):
+        assert m.moe_get_device_error(L.ws) == 0
+        xin = lays[0]["x"] if l == 0 else ys[l - 1].view(torch.int16).cpu().numpy().view(np.uint16)
+        ref = dict(lay, x=np.ascontiguousarray(xin))
+        out = dict(y=ys[l].float().cpu().numpy().astype(np.float64), idx=L.topk_idx[:T].cpu().numpy())
+        check_output(out, ref, np.arange(T))
+        y_ref, idx_ref, _ = oracle.layer(ref)
+        assert np.array_equal(out["idx"], idx_ref), "layer %d routing differs" % l
