@@ -7,7 +7,9 @@ Default workload: decode, T = 1 token through 40 distinct seeded layers
 packed weights resident and cycled, so every step streams its weights from
 HBM (inputs larger than L2; no flush needed).  One step = the whole hot path
 (route, permute, expert FFN, combine) of all 40 layers, replayed as one CUDA
-graph.  A second, smaller measurement covers the T = 2048 prefill layer.
+graph.  A second, smaller measurement covers the T = 2048 prefill layer, and
+a report-only one the T = 8 (H 512), T = 512 Zipf-skewed and T = 16384
+hot-expert layers (``other_configs``, L2 flushed between iterations).
 
 Prints one JSON line on rank 0.  Under torchrun every rank runs its own
 replica (weak scaling, no collective on the data path); the time is the max
@@ -410,6 +412,89 @@ def run_prefill(device, steps, warmup, world, peaks):
             "l2": "inputs larger than L2 (455.8 MB of packed weights per layer)"}
 
 
+def expert_bytes(h: int, i: int, g: int = G) -> int:
+    """Packed bytes of one expert: gate/up [2i, h] and down [h, i] 4-bit codes
+    plus one bf16 (scale, bias) pair per group of g inputs."""
+    return (2 * i * h + h * i) // 2 + (2 * i * (h // g) + h * (i // g)) * 4
+
+
+def _timed_flushed(replay, n, stream, flush):
+    """Device time (ms) of n calls of replay(), each bracketed by its own CUDA
+    events on stream, with flush() (an L2-sized write) between them outside
+    the events."""
+    import torch
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    torch.cuda.synchronize()
+    for s, e in ev:
+        flush()
+        s.record(stream)
+        replay()
+        e.record(stream)
+    torch.cuda.synchronize()
+    return sum(s.elapsed_time(e) for s, e in ev)
+
+
+def run_other_configs(device, steps, warmup, peaks, ids=(0, 2, 4)):
+    """Report-only layer measurements of the remaining synthetic workloads:
+    the T=8 small case (H 512, I 128), the Zipf-skewed T=512 layer and the
+    T=16384 layer with half its tokens biased onto 8 hot experts.  Scatter
+    mode, the default implementation path, L2 flushed between iterations.
+    Each reports layer tokens/s, the expert-FFN time, its HBM fraction on the
+    bytes of the experts the routing activated and its bf16 tensor fraction."""
+    import torch
+    import gen
+    from bit_dequant_expert_b200 import MOE_MODE_SCATTER
+    from bit_dequant_expert_b200.layer import MoELayer, to_device
+    import bit_dequant_expert_b200 as m
+    stream = torch.cuda.Stream(device=device)
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    out = {}
+    for cid in ids:
+        spec = gen.config(cid)
+        lay = gen.make_layer(spec)
+        T, h, i = spec.T, spec.H, spec.I
+        L = MoELayer(lay, max_tokens=T, device=device, mode=MOE_MODE_SCATTER)
+        x = to_device(lay["x"], device)
+        bias = lay["logit_bias"]
+        stride = int(lay["bias_stride"])
+        bias_t = None if bias is None else to_device(bias, device)
+        del lay
+
+        def fwd():
+            L.forward(x, logit_bias=bias_t, bias_stride=stride)
+
+        def ffn():
+            L.expert_ffn(x, T)
+
+        with torch.cuda.stream(stream):
+            fwd()
+        torch.cuda.synchronize()
+        err = m.moe_get_device_error(L.ws)
+        active = int((L.counts > 0).sum().item())
+        g_fwd, g_ffn = _capture(fwd, stream), _capture(ffn, stream)
+        with torch.cuda.stream(stream):
+            for _ in range(warmup):
+                g_fwd.replay()
+                g_ffn.replay()
+            flush = lambda: flush_buf.zero_()
+            ms = _timed_flushed(g_fwd.replay, steps, stream, flush) / steps
+            ffn_ms = _timed_flushed(g_ffn.replay, steps, stream, flush) / steps
+        rows = (K + 1) * T
+        flops = 2.0 * rows * (2 * i * h + h * i)
+        wbytes = (active + 1) * expert_bytes(h, i)
+        out[str(cid)] = {
+            "workload": spec.name, "T": T, "value": T / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
+            "ffn_ms": ffn_ms, "steps": steps, "device_error": err, "active_experts": active,
+            "hbm_frac_active_weight_bytes": wbytes / (ffn_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+            "tensor_frac": flops / (ffn_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+            "algorithmic_flops": flops, "active_weight_bytes": wbytes,
+            "gpu_launches_per_step": _launch_count(L, T),
+            "l2": "flushed between timed iterations (256 MB write outside the events)"}
+        del L, x, bias_t, g_fwd, g_ffn
+        torch.cuda.synchronize()
+    return out
+
+
 def run_ncu_case(case, device, calls):
     """One layer for a profiler: route + permute, then `calls` launches of the kernel under study."""
     import torch
@@ -450,6 +535,9 @@ def main(argv=None):
                          "--steps calls of the named kernel (decode: config 1 layer 0, T=1; prefill: "
                          "config 3, T=2048); prints the device error word and nothing timed")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle CPU baseline")
+    ap.add_argument("--other-configs", choices=("on", "off", "only"), default="on",
+                    help="report-only layer measurements of the T=8 (H 512), T=512 Zipf and T=16384 hot-expert "
+                         "workloads: 'on' adds them to the line as other_configs, 'only' prints just them")
     args = ap.parse_args(argv)
     warmup = max(args.warmup, 3)
     world, rank, local = dist_env()
@@ -468,6 +556,16 @@ def main(argv=None):
 
     if args.ncu_case:
         return run_ncu_case(args.ncu_case, device, max(args.steps, 1))
+
+    if args.other_configs == "only":
+        oc = run_other_configs(device, max(args.steps // 10, 5), warmup, peaks)
+        if rank == 0:
+            print(json.dumps({"other_configs": oc, "peaks": peaks}), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            barrier(world)
+            dist.destroy_process_group()
+        return 0
 
     if args.prefill_only:
         pre = run_prefill(device, max(args.steps, 1), warmup, world, peaks)
@@ -527,6 +625,8 @@ def main(argv=None):
     }
     if pre is not None:
         line["prefill_t2048"] = pre
+    if args.other_configs == "on":
+        line["other_configs"] = run_other_configs(device, max(args.steps // 10, 5), warmup, peaks)
     if rank == 0 and world == 1:
         budget = args.cpu_budget
         layers_host = res.pop("_host_layers")
