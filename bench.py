@@ -213,6 +213,52 @@ def time_oracle_decode(layers: list, budget_s: float):
     return done / dt, done, dt
 
 
+def _omp_set_threads(n: int) -> None:
+    import ctypes
+    ctypes.CDLL("libgomp.so.1").omp_set_num_threads(int(n))
+
+
+def time_oracle_layer(lay: dict, budget_s: float):
+    """Tokens/s of the oracle on a prefix of the layer's tokens (with its
+    logit bias): the prefix doubles from 1 token while the next call is
+    expected to fit in budget_s; returns (rate, tokens, seconds) of the last
+    call."""
+    import oracle
+    T = lay["x"].shape[0]
+    n, spent, last = 1, 0.0, None
+    while True:
+        tok = np.arange(n, dtype=np.int32)
+        t0 = time.perf_counter()
+        oracle.layer(lay, tokens=tok)
+        dt = time.perf_counter() - t0
+        spent += dt
+        last = (n / dt, n, dt)
+        if n >= T or spent + 2.2 * dt > budget_s:
+            return last
+        n = min(2 * n, T)
+
+
+def time_oracle_other_configs(budget_s: float, ids=(0, 2, 4), single_thread=(0, 2)):
+    """The oracle's layer tokens/s on each configuration, on all OpenMP
+    threads and, for the smaller ones, on one thread."""
+    import gen
+    out = {}
+    full = omp_threads()
+    for cid in ids:
+        lay = gen.make_layer(gen.config(cid))
+        runs = [("all", full)] + ([("1", 1)] if cid in single_thread else [])
+        out[str(cid)] = {}
+        for label, nt in runs:
+            _omp_set_threads(nt)
+            try:
+                rate, n, dt = time_oracle_layer(lay, budget_s)
+            finally:
+                _omp_set_threads(full)
+            out[str(cid)][label] = {"value": rate, "unit": UNIT, "cores": nt, "kind": "oracle",
+                                    "sample": "first %d of %d tokens in one call, %.2f s" % (n, lay["x"].shape[0], dt)}
+    return out
+
+
 # ------------------------------------------------------------- workloads
 
 
@@ -633,6 +679,9 @@ def main(argv=None):
         rate, n, dt = time_oracle_decode(layers_host, budget)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": omp_threads(), "kind": "oracle",
                                 "sample": "%d layer passes (T=1) of the first decode layers, %.1f s" % (n, dt)}
+        if "other_configs" in line:
+            for cid, cpu in time_oracle_other_configs(budget / 4).items():
+                line["other_configs"][cid]["cpu_baseline"] = cpu
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

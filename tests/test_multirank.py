@@ -66,3 +66,17 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     monkeypatch.setenv("WORLD_SIZE", "2")
     assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3"]) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_oracle_timing_per_config_restores_threads():
+    """The per-configuration oracle baseline: a bounded token prefix, one
+    thread where asked, and the OpenMP thread count put back afterwards."""
+    sys.path.insert(0, ROOT)
+    import bench
+    before = bench.omp_threads()
+    out = bench.time_oracle_other_configs(0.3, ids=(0,), single_thread=(0,))
+    assert bench.omp_threads() == before
+    assert set(out["0"]) == {"all", "1"}
+    assert out["0"]["1"]["cores"] == 1 and out["0"]["all"]["cores"] == before
+    for run in out["0"].values():
+        assert run["kind"] == "oracle" and run["value"] > 0 and "of 8 tokens" in run["sample"]
