@@ -43,7 +43,7 @@ MOE_PATH_TC = 3
 EXPORTED = (
     "moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permute", "moe_expert_ffn",
     "moe_expert_ffn_path", "moe_combine", "moe_get_device_error", "moe_status_string", "moe_launch_count",
-    "moe_permute_static", "moe_decode_layer",
+    "moe_permute_static", "moe_decode_layer", "moe_wait_selftest",
 )
 
 MOE_STATIC_MAX_TOKENS = 16384
@@ -88,6 +88,8 @@ _lib.moe_launch_count.restype = _I32
 _lib.moe_launch_count.argtypes = [_CFG, _I32, _I32, _I32]
 _lib.moe_status_string.restype = ctypes.c_char_p
 _lib.moe_status_string.argtypes = [_I32]
+_lib.moe_wait_selftest.restype = _I32
+_lib.moe_wait_selftest.argtypes = [_I32, _I32, _I32, ctypes.c_uint64, _P, _P]
 
 
 class MoeError(RuntimeError):
@@ -205,6 +207,15 @@ def moe_launch_count(cfg, T, mode=MOE_MODE_SCATTER, path=MOE_PATH_AUTO) -> int:
 
 def moe_get_device_error(ws, stream=None) -> int:
     return int(_lib.moe_get_device_error(_ptr(ws), _stream(stream)))
+
+
+def moe_wait_selftest(kind: int, ctas: int, skip_cta: int, limit_ns: int, ws, stream=None,
+                      raise_on_error=True) -> int:
+    """Makes a bounded device wait expire on purpose (kind 0: an mbarrier
+    nothing arrives on; kind 1: a grid barrier of `ctas` CTAs without CTA
+    `skip_cta`'s arrival); read the outcome with moe_get_device_error(ws)."""
+    st = _lib.moe_wait_selftest(kind, ctas, skip_cta, limit_ns, _ptr(ws), _stream(stream))
+    return _check(st, "moe_wait_selftest", raise_on_error)
 
 
 from .layer import MoELayer  # noqa: E402  (torch-level convenience wrapper)

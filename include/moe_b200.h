@@ -239,6 +239,32 @@ int32_t moe_launch_count(const moe_config_t* cfg, int32_t T, int32_t mode, int32
 /* Human-readable name of a status code (static string). */
 const char* moe_status_string(int32_t status);
 
+/*
+ * moe_wait_selftest: failure-detection self-test.  The Lily pages have no
+ * counterpart; it exists so that a caller (a test, a health check) can make
+ * one of the library's bounded device waits expire on purpose and confirm
+ * that the expiry is reported and that the context stays usable.  It
+ * computes nothing.
+ *   kind 0     one thread waits on a shared-memory mbarrier that nothing
+ *              arrives on (the pipeline wait of the FFN kernels); ctas must
+ *              be 1 and skip_cta -1.  Always ends in MOE_ERR_TIMEOUT.
+ *   kind 1     ctas CTAs (1..148) meet at a grid barrier on a 64-bit counter
+ *              (the decode kernels' barrier); the arrival of CTA skip_cta is
+ *              suppressed, so the others' waits expire (MOE_ERR_TIMEOUT);
+ *              skip_cta = -1 suppresses none and the barrier completes with
+ *              no error.
+ *   limit_ns   how long each wait lasts before it gives up: 1e3..1e9 ns.
+ *   ws         a workspace (256-byte aligned, at least 256 bytes): the
+ *              timeout goes to its sticky error word, read it with
+ *              moe_get_device_error.  The call also clears and uses 8
+ *              reserved bytes of the workspace header for the counter;
+ *              nothing else in the workspace is touched.
+ * Asynchronous on stream.  Returns MOE_ERR_WORKSPACE for a null or
+ * misaligned ws, MOE_ERR_INVALID_ARG for any other bad argument (nothing is
+ * launched), MOE_ERR_CUDA if the launch fails, else MOE_OK.
+ */
+int32_t moe_wait_selftest(int32_t kind, int32_t ctas, int32_t skip_cta, uint64_t limit_ns, void* ws, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -103,6 +103,28 @@ def test_decode_layer_validation_before_launch():
     assert _decode(cfg, 8, need, bias=FAKE, stride=-1) == m.MOE_ERR_INVALID_ARG
 
 
+def test_wait_selftest_validation_before_launch():
+    """The failure-detection self-test refuses a bad kind, CTA count,
+    suppressed CTA, wait limit or workspace before launching anything."""
+    import bit_dequant_expert_b200 as m
+
+    def call(kind=1, ctas=4, skip=1, limit=1_000_000, ws=FAKE):
+        return m.moe_wait_selftest(kind, ctas, skip, limit, ws, stream=0, raise_on_error=False)
+
+    assert call(ws=None) == m.MOE_ERR_WORKSPACE
+    assert call(ws=FAKE + 16) == m.MOE_ERR_WORKSPACE
+    assert call(kind=2) == m.MOE_ERR_INVALID_ARG
+    assert call(kind=-1) == m.MOE_ERR_INVALID_ARG
+    assert call(kind=0, ctas=2, skip=-1) == m.MOE_ERR_INVALID_ARG
+    assert call(kind=0, ctas=1, skip=0) == m.MOE_ERR_INVALID_ARG
+    assert call(ctas=0, skip=-1) == m.MOE_ERR_INVALID_ARG
+    assert call(ctas=149, skip=-1) == m.MOE_ERR_INVALID_ARG
+    assert call(ctas=4, skip=4) == m.MOE_ERR_INVALID_ARG
+    assert call(ctas=4, skip=-2) == m.MOE_ERR_INVALID_ARG
+    assert call(limit=999) == m.MOE_ERR_INVALID_ARG
+    assert call(limit=1_000_000_001) == m.MOE_ERR_INVALID_ARG
+
+
 def test_launch_count_per_path():
     """Kernels per layer as the bench counts them (host-only, no device needed)."""
     import bit_dequant_expert_b200 as m
