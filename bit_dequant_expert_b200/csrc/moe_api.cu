@@ -55,7 +55,8 @@ int32_t* err_word(void* ws) { return reinterpret_cast<int32_t*>(ws); }
 int32_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 // Implementation chosen for MOE_PATH_AUTO: the memory-bound decode kernel for
-// a handful of tokens, otherwise the general CUDA-core path.
+// a handful of tokens, else the tensor-core kernel where its shape rules
+// hold, else the CUDA-core path.
 int32_t resolve_path(const FfnArgs& a) {
     if (ffn_gemv_supported(a)) return MOE_PATH_GEMV;
     if (ffn_tc_supported(a)) return MOE_PATH_TC;

@@ -84,7 +84,7 @@ typedef struct {
 #define MOE_PATH_AUTO 0
 #define MOE_PATH_SIMT 1    /* CUDA-core dequant + dot products, any T */
 #define MOE_PATH_GEMV 2    /* memory-bound split-K GEMV, few rows per expert */
-#define MOE_PATH_TC 3      /* TMA + in-smem dequant + tcgen05 MMA into TMEM */
+#define MOE_PATH_TC 3      /* TMA; dequant in registers into tensor memory (A); tcgen05 MMA */
 
 /* Bytes of workspace that the calls need for up to max_tokens tokens; 0 if
  * the configuration is unsupported.  Caller allocates it (256-byte aligned)
