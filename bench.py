@@ -45,10 +45,6 @@ FFN_BYTES_T1 = 9 * EXPERT_BYTES + H * 2 + H * 4      # + x (bf16) + y_acc (fp32)
 LAYER_BYTES_T1 = FFN_BYTES_T1 + ROUTER_BYTES
 
 
-def log(*a):
-    print(*a, file=sys.stderr, flush=True)
-
-
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):

@@ -4,7 +4,6 @@ from __future__ import annotations
 
 import numpy as np
 
-import gen
 import oracle
 
 ROW_REL_TOL = 1e-2       # per token: max_h |y_gpu - y_ref| / max_h |y_ref|

@@ -5,7 +5,6 @@ Mutants are built from a patched copy of oracle/moe_oracle.c in a temporary
 directory; the real oracle is never touched.
 """
 import os
-import shutil
 import subprocess
 
 import pytest
