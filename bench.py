@@ -563,6 +563,45 @@ def run_ncu_case(case, device, calls):
     return 0
 
 
+DECODE_WORKLOAD = "decode: T=1 x 40 distinct layers cycled (H 2048, I 512, E 256 top-8 + shared, G 64)"
+
+
+def decode_line(res: dict, ms: float, units: float, world: int, steps: int, warmup: int, peaks: dict) -> dict:
+    """The JSON line of the decode measurement: `ms` is the slowest rank's
+    time per step, `units` the layer passes all ranks made per step, `res`
+    what run_decode measured."""
+    return {
+        "metric": METRIC,
+        "value": units / (ms / 1e3),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": steps,
+        "warmup": warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16 (4-bit weights, fp32 accumulation)",
+        "data": "synthetic (seeded; SplitMix64 layers shaped like the pages' model)",
+        "config": {
+            "workload": DECODE_WORKLOAD,
+            "global_batch": world,
+            "seq_len": 1,
+            "parallelism": "replicas" if world > 1 else "single GPU",
+            "l2": "inputs larger than L2 (18.2 GB of weights streamed per step; no flush)",
+            "graph": "one CUDA graph per step (40 layers x moe_decode_layer: fused route + permute + expert FFN kernel, then combine)",
+        },
+        "decode_token_per_s": world / (ms / 1e3),
+        "breakdown_us_per_layer": res["breakdown_us_per_layer"],
+        "gpu_launches": res["gpu_launches"],
+        "roofline": res["roofline"],
+        "roofline_layer": res["roofline_layer"],
+        "e2e": res["e2e"],
+        "clocks": res["clocks"],
+        "peaks": peaks,
+    }
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -633,38 +672,7 @@ def main(argv=None):
     pre = None if args.no_prefill else run_prefill(device, max(args.steps // 10, 5), warmup, world, peaks)
 
     ms, units = aggregate(res["ms_per_step"], res["units_per_step"], world)
-    value = units / (ms / 1e3)
-
-    line = {
-        "metric": METRIC,
-        "value": value,
-        "unit": UNIT,
-        "n_gpus": world,
-        "steps": args.steps,
-        "warmup": warmup,
-        "ms_per_step": ms,
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": "bf16 (4-bit weights, fp32 accumulation)",
-        "data": "synthetic (seeded; SplitMix64 layers shaped like the pages' model)",
-        "config": {
-            "workload": "decode: T=1 x 40 distinct layers cycled (H 2048, I 512, E 256 top-8 + shared, G 64)",
-            "global_batch": world,
-            "seq_len": 1,
-            "parallelism": "replicas" if world > 1 else "single GPU",
-            "l2": "inputs larger than L2 (18.2 GB of weights streamed per step; no flush)",
-            "graph": "one CUDA graph per step (40 layers x moe_decode_layer: fused route + permute + expert FFN kernel, then combine)",
-        },
-        "decode_token_per_s": world / (ms / 1e3),
-        "breakdown_us_per_layer": res["breakdown_us_per_layer"],
-        "gpu_launches": res["gpu_launches"],
-        "roofline": res["roofline"],
-        "roofline_layer": res["roofline_layer"],
-        "e2e": res["e2e"],
-        "clocks": res["clocks"],
-        "peaks": peaks,
-    }
+    line = decode_line(res, ms, units, world, args.steps, warmup, peaks)
     if pre is not None:
         line["prefill_t2048"] = pre
     if args.other_configs == "on":
@@ -711,8 +719,7 @@ def run_reference(args, world, rank, warmup):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": len(per_step),
         "warmup": warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic (seeded)",
-        "config": {"workload": "decode: T=1 x 40 distinct layers cycled (H 2048, I 512, E 256 top-8 + shared, G 64)",
-                   "global_batch": 1, "seq_len": 1, "parallelism": "host cores"},
+        "config": {"workload": DECODE_WORKLOAD, "global_batch": 1, "seq_len": 1, "parallelism": "host cores"},
         "impl": "reference",
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": omp_threads(), "kind": "oracle",
                          "sample": "one layer pass (T=1) per step, layers 0-2 cycled"},
