@@ -476,13 +476,29 @@ def _timed_flushed(replay, n, stream, flush):
     return sum(s.elapsed_time(e) for s, e in ev)
 
 
-def run_other_configs(device, steps, warmup, peaks, ids=(0, 2, 4)):
-    """Report-only layer measurements of the remaining synthetic workloads:
-    the T=8 small case (H 512, I 128), the Zipf-skewed T=512 layer and the
-    T=16384 layer with half its tokens biased onto 8 hot experts.  Scatter
-    mode, the default implementation path, L2 flushed between iterations.
-    Each reports layer tokens/s, the expert-FFN time, its HBM fraction on the
-    bytes of the experts the routing activated and its bf16 tensor fraction."""
+def other_config_specs() -> dict:
+    """The remaining synthetic workloads, each (layer spec, layer index): the
+    T=8 small case (H 512, I 128), the Zipf-skewed T=512 layer and the
+    T=16384 layer with half its tokens biased onto 8 hot experts."""
+    import gen
+    return {str(c): (gen.config(c), 0) for c in (0, 2, 4)}
+
+
+def small_t_specs() -> dict:
+    """Decode-layer shapes (H 2048, I 512) with a few tokens, as speculative
+    decoding's verification batches: 2-8 tokens through the decode kernel
+    (weights read = the union of the selected experts), and 16 tokens, past
+    the crossover to the tensor-core kernel."""
+    import gen
+    return {"T%d" % t: (gen.config(1).with_T(t), 3) for t in (2, 4, 8, 16)}
+
+
+def run_other_configs(device, steps, warmup, peaks, specs=None):
+    """Report-only layer measurements of `specs` (default: other_config_specs()).
+    Scatter mode, the default implementation path, L2 flushed between
+    iterations.  Each reports layer tokens/s, the expert-FFN time, its HBM
+    fraction on the bytes of the experts the routing activated (with the
+    shared expert) and its bf16 tensor fraction."""
     import torch
     import gen
     from bit_dequant_expert_b200 import MOE_MODE_SCATTER
@@ -491,9 +507,8 @@ def run_other_configs(device, steps, warmup, peaks, ids=(0, 2, 4)):
     stream = torch.cuda.Stream(device=device)
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=device)
     out = {}
-    for cid in ids:
-        spec = gen.config(cid)
-        lay = gen.make_layer(spec)
+    for cid, (spec, layer_index) in (specs or other_config_specs()).items():
+        lay = gen.make_layer(spec, layer_index)
         T, h, i = spec.T, spec.H, spec.I
         L = MoELayer(lay, max_tokens=T, device=device, mode=MOE_MODE_SCATTER)
         x = to_device(lay["x"], device)
@@ -524,9 +539,9 @@ def run_other_configs(device, steps, warmup, peaks, ids=(0, 2, 4)):
         rows = (K + 1) * T
         flops = 2.0 * rows * (2 * i * h + h * i)
         wbytes = (active + 1) * expert_bytes(h, i)
-        out[str(cid)] = {
-            "workload": spec.name, "T": T, "value": T / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
-            "ffn_ms": ffn_ms, "steps": steps, "device_error": err, "active_experts": active,
+        out[cid] = {
+            "workload": "%s (T=%d, layer %d)" % (spec.name, T, layer_index), "T": T,
+            "value": T / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms, "ffn_ms": ffn_ms, "steps": steps, "device_error": err, "active_experts": active,
             "hbm_frac_active_weight_bytes": wbytes / (ffn_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
             "tensor_frac": flops / (ffn_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
             "algorithmic_flops": flops, "active_weight_bytes": wbytes,
@@ -618,7 +633,8 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle CPU baseline")
     ap.add_argument("--other-configs", choices=("on", "off", "only"), default="on",
                     help="report-only layer measurements of the T=8 (H 512), T=512 Zipf and T=16384 hot-expert "
-                         "workloads: 'on' adds them to the line as other_configs, 'only' prints just them")
+                         "workloads, and of decode-layer shapes with 2-16 tokens: 'on' adds them to the line "
+                         "(other_configs, small_t), 'only' prints just them")
     args = ap.parse_args(argv)
     warmup = max(args.warmup, 3)
     world, rank, local = dist_env()
@@ -640,8 +656,9 @@ def main(argv=None):
 
     if args.other_configs == "only":
         oc = run_other_configs(device, max(args.steps // 10, 5), warmup, peaks)
+        st = run_other_configs(device, max(args.steps // 10, 5), warmup, peaks, small_t_specs())
         if rank == 0:
-            print(json.dumps({"other_configs": oc, "peaks": peaks}), flush=True)
+            print(json.dumps({"other_configs": oc, "small_t": st, "peaks": peaks}), flush=True)
         if world > 1:
             import torch.distributed as dist
             barrier(world)
@@ -677,6 +694,7 @@ def main(argv=None):
         line["prefill_t2048"] = pre
     if args.other_configs == "on":
         line["other_configs"] = run_other_configs(device, max(args.steps // 10, 5), warmup, peaks)
+        line["small_t"] = run_other_configs(device, max(args.steps // 10, 5), warmup, peaks, small_t_specs())
     if rank == 0 and world == 1:
         budget = args.cpu_budget
         layers_host = res.pop("_host_layers")

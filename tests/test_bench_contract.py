@@ -74,3 +74,14 @@ def test_reference_arm_line(monkeypatch, capsys):
     assert cpu["kind"] == "oracle" and cpu["cores"] >= 1 and cpu["value"] == line["value"] and cpu["sample"]
     assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
+
+
+def test_report_only_workloads():
+    """The report-only layers: configurations 0, 2 and 4 as the generator
+    defines them, and decode-layer shapes at 2, 4, 8 and 16 tokens."""
+    other = bench.other_config_specs()
+    assert sorted(other) == ["0", "2", "4"]
+    assert [(other[k][0].T, other[k][0].H) for k in ("0", "2", "4")] == [(8, 512), (512, 2048), (16384, 2048)]
+    small = bench.small_t_specs()
+    assert {k: (s.T, s.H, s.I, s.E) for k, (s, _) in small.items()} == {
+        "T2": (2, 2048, 512, 256), "T4": (4, 2048, 512, 256), "T8": (8, 2048, 512, 256), "T16": (16, 2048, 512, 256)}
