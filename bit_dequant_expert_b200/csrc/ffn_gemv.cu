@@ -14,7 +14,8 @@
 //    of H, keeps those 32 h values in shared memory, and multiplies them by
 //    the matching 32 columns of the down matrix for every output row
 //    (split-K over the intermediate size), adding w * y into y_acc.  No CTA
-//    waits for another.
+//    waits for another's compute; only the first addition into y_acc waits
+//    until every CTA has cleared its slice of it (last point below).
 //  - A producer warp moves each unit in a few large TMA boxes: gate and up
 //    codes of 8 of the 32 rows per box, whole rows (16 KB: two contiguous
 //    8 KB runs of HBM; 128B-swizzled so the consumers' 16-byte reads hit
