@@ -26,6 +26,22 @@ def to_device(a, device, dtype=None) -> torch.Tensor:
     return t.to(device)
 
 
+def check_rows(t, name: str, H: int, device: torch.device) -> None:
+    """Raises unless t is a contiguous bf16 [n, H] tensor on `device` (any
+    index of its type when `device` names none): the library reads it through
+    its data pointer alone."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor, got %s" % (name, type(t).__name__))
+    if t.dtype != torch.bfloat16:
+        raise TypeError("%s must be bfloat16, got %s" % (name, t.dtype))
+    if t.dim() != 2 or t.shape[1] != H:
+        raise ValueError("%s must have shape [T, %d], got %s" % (name, H, tuple(t.shape)))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if t.device.type != device.type or (device.index is not None and t.device.index != device.index):
+        raise ValueError("%s is on %s, the layer on %s" % (name, t.device, device))
+
+
 class MoELayer:
     """One layer's weights resident on the device plus its scratch buffers.
 
@@ -94,9 +110,14 @@ class MoELayer:
                 y_out=None) -> torch.Tensor:
         """y [T, H] bf16 for x [T, H] bf16 (written to y_out if given, else to
         the layer's own output buffer, a view of which is returned)."""
+        check_rows(x, "x", self.H, self.device)
         T = x.shape[0]
         if T > self.max_tokens:
             raise ValueError("T=%d exceeds max_tokens=%d" % (T, self.max_tokens))
+        if y_out is not None:
+            check_rows(y_out, "y_out", self.H, self.device)
+            if y_out.shape[0] < T:
+                raise ValueError("y_out has %d rows, fewer than the %d tokens" % (y_out.shape[0], T))
         if self.fused_ok(T) and logits_in is None:
             return self.decode_fused(x, T, logit_bias, bias_stride, stream, y_out)
         self.route(x, T, logit_bias, bias_stride, logits_in, stream)
