@@ -42,6 +42,21 @@ def check_rows(t, name: str, H: int, device: torch.device) -> None:
         raise ValueError("%s is on %s, the layer on %s" % (name, t.device, device))
 
 
+def check_f32(t, name: str, min_numel: int, device: torch.device) -> None:
+    """Raises unless t is a contiguous fp32 tensor of at least min_numel
+    elements on `device`."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor, got %s" % (name, type(t).__name__))
+    if t.dtype != torch.float32:
+        raise TypeError("%s must be float32, got %s" % (name, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if t.numel() < min_numel:
+        raise ValueError("%s has %d elements, fewer than the %d read" % (name, t.numel(), min_numel))
+    if t.device.type != device.type or (device.index is not None and t.device.index != device.index):
+        raise ValueError("%s is on %s, the layer on %s" % (name, t.device, device))
+
+
 class MoELayer:
     """One layer's weights resident on the device plus its scratch buffers.
 
@@ -118,6 +133,12 @@ class MoELayer:
             check_rows(y_out, "y_out", self.H, self.device)
             if y_out.shape[0] < T:
                 raise ValueError("y_out has %d rows, fewer than the %d tokens" % (y_out.shape[0], T))
+        if logit_bias is not None:
+            if bias_stride < 0:
+                raise ValueError("bias_stride must be >= 0, got %d" % bias_stride)
+            check_f32(logit_bias, "logit_bias", (T - 1) * bias_stride + self.E, self.device)
+        if logits_in is not None:
+            check_f32(logits_in, "logits_in", T * self.E, self.device)
         if self.fused_ok(T) and logits_in is None:
             return self.decode_fused(x, T, logit_bias, bias_stride, stream, y_out)
         self.route(x, T, logit_bias, bias_stride, logits_in, stream)

@@ -61,4 +61,15 @@ def test_forward_checks_before_any_call():
         L.forward(x, y_out=torch.zeros(2, H, dtype=torch.bfloat16))  # too few output rows
     with pytest.raises(TypeError):
         L.forward(x, y_out=torch.zeros(3, H, dtype=torch.float32))
+    with pytest.raises(TypeError):
+        L.forward(x, logit_bias=torch.zeros(256, dtype=torch.bfloat16))
+    with pytest.raises(ValueError):
+        L.forward(x, logit_bias=torch.zeros(2, 256), bias_stride=256)      # 3 tokens need 3 rows
+    with pytest.raises(ValueError):
+        L.forward(x, logit_bias=torch.zeros(256), bias_stride=-1)
+    with pytest.raises(ValueError):
+        L.forward(x, logits_in=torch.zeros(2, 256))
     assert calls == []
+    L.forward(x, logit_bias=torch.zeros(256))                              # one row for every token
+    L.forward(x, logit_bias=torch.zeros(3, 256), bias_stride=256)          # one row per token
+    assert calls == [("fused", 3), ("fused", 3)]
