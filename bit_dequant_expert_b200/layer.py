@@ -57,6 +57,37 @@ def check_f32(t, name: str, min_numel: int, device: torch.device) -> None:
         raise ValueError("%s is on %s, the layer on %s" % (name, t.device, device))
 
 
+_BF16_BITS = (np.dtype(np.uint16), torch.bfloat16, torch.int16)
+_CODE_WORDS = (np.dtype(np.uint32), torch.int32, torch.uint32)
+
+
+def check_weights(weights: dict, group_size: int = 64) -> tuple:
+    """(E, H, I) of a packed layer, after checking that every array has the
+    shape and element type the library reads it with (bf16 bits for w_router
+    and the (scale, bias) pairs, 32-bit words for the codes); raises
+    ValueError or TypeError otherwise."""
+    for name in ("w_router", "gu_codes", "gu_sb", "d_codes", "d_sb"):
+        if name not in weights:
+            raise ValueError("weights lack %s" % name)
+    gu = weights["gu_codes"]
+    if len(gu.shape) != 3:
+        raise ValueError("gu_codes must be [E+1, 2I, H/8], got %s" % (tuple(gu.shape),))
+    E1, I2, H8 = (int(v) for v in gu.shape)
+    E, H, I, G = E1 - 1, 8 * H8, I2 // 2, group_size
+    if E < 1 or I2 % 2 or H % G or I % G:
+        raise ValueError("gu_codes shape %s gives no layer with groups of %d" % (tuple(gu.shape), G))
+    want = {"w_router": (E, H), "gu_codes": (E1, 2 * I, H // 8), "gu_sb": (E1, 2 * I, H // G, 2),
+            "d_codes": (E1, H, I // 8), "d_sb": (E1, H, I // G, 2)}
+    for name, shape in want.items():
+        got = tuple(int(v) for v in weights[name].shape)
+        if got != shape:
+            raise ValueError("%s must have shape %s, got %s" % (name, shape, got))
+        kinds = _CODE_WORDS if name.endswith("codes") else _BF16_BITS
+        if weights[name].dtype not in kinds:
+            raise TypeError("%s has element type %s" % (name, weights[name].dtype))
+    return E, H, I
+
+
 class MoELayer:
     """One layer's weights resident on the device plus its scratch buffers.
 
@@ -67,10 +98,8 @@ class MoELayer:
 
     def __init__(self, weights: dict, max_tokens: int, device="cuda", mode=MOE_MODE_SCATTER,
                  path=MOE_PATH_AUTO, has_shared=True):
-        gu = weights["gu_codes"]
-        E1, I2, H8 = gu.shape
-        H = H8 * 8
-        I = I2 // 2
+        E, H, I = check_weights(weights)
+        E1 = E + 1
         self.cfg = config(hidden=H, inter=I, num_experts=E1 - 1, top_k=8, group_size=64,
                           has_shared=1 if has_shared else 0)
         self.H, self.I, self.E, self.K = H, I, E1 - 1, 8

@@ -73,3 +73,24 @@ def test_forward_checks_before_any_call():
     L.forward(x, logit_bias=torch.zeros(256))                              # one row for every token
     L.forward(x, logit_bias=torch.zeros(3, 256), bias_stride=256)          # one row per token
     assert calls == [("fused", 3), ("fused", 3)]
+
+
+def test_check_weights():
+    import numpy as np
+    import gen
+    from bit_dequant_expert_b200.layer import check_weights
+    lay = gen.make_weights(gen.config(0))
+    assert check_weights(lay) == (256, 512, 128)
+    assert check_weights(gen.make_weights(gen.LayerSpec(T=1, H=1024, I=256))) == (256, 1024, 256)
+    as_tensors = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16) if v.dtype == np.uint16
+                  else torch.from_numpy(v.view(np.int32)) for k, v in lay.items()}
+    assert check_weights(as_tensors) == (256, 512, 128)
+    bad = [("d_codes", lay["d_codes"][:, :-8]), ("gu_sb", lay["gu_sb"][:, :, :-1]),
+           ("w_router", lay["w_router"][:-1]), ("d_sb", lay["d_sb"].astype(np.float32))]
+    for name, arr in bad:
+        with pytest.raises((ValueError, TypeError)):
+            check_weights(dict(lay, **{name: arr}))
+    with pytest.raises(ValueError):
+        check_weights({k: v for k, v in lay.items() if k != "d_sb"})
+    with pytest.raises(TypeError):
+        check_weights(dict(lay, w_router=lay["w_router"].astype(np.float32)))
