@@ -77,13 +77,14 @@ def check_permutation_props(out, T, E=256, K=8):
     assert np.array_equal(e_of_row, np.repeat(np.arange(E), counts))
 
 
-def check_output(out, lay, tokens, T=None, logits_in=None, tol=ROW_REL_TOL):
+def check_output(out, lay, tokens, T=None, logits_in=None, tol=ROW_REL_TOL, has_shared=True):
     T = T or lay["x"].shape[0]
     sub = dict(lay)
     sub["x"] = lay["x"][:T]
     if lay.get("logit_bias") is not None and int(lay.get("bias_stride", 0)):
         sub["logit_bias"] = lay["logit_bias"][:T]
-    y_ref, idx_ref, _ = oracle.layer(sub, tokens=np.asarray(tokens, dtype=np.int32), logits_in=logits_in)
+    y_ref, idx_ref, _ = oracle.layer(sub, tokens=np.asarray(tokens, dtype=np.int32), logits_in=logits_in,
+                                     has_shared=has_shared)
     err = row_rel_err(out["y"][tokens], y_ref)
     assert err.max() <= tol, "max row-relative error %.3e (token %d)" % (err.max(), int(np.argmax(err)))
     return err

@@ -288,28 +288,6 @@ def test_fused_decode_layers():
         _fused_vs_oracle(gen.make_layer(spec, layer), 1)
 
 
-@pytest.mark.parametrize("T", [2, 4, 5, 8])
-def test_fused_decode_verification_batches(T):
-    """Decode-layer shapes (H 2048, I 512) with 2-8 tokens, as a verification
-    batch of speculative decoding sends them: the weights read are those of
-    the union of the experts the tokens select."""
-    _fused_vs_oracle(gen.make_layer(gen.config(1).with_T(T), 3), T)
-
-
-def test_decode_shape_past_the_crossover():
-    """16 tokens at decode-layer shapes take the four calls with the
-    tensor-core expert FFN (scatter mode): routing bit-exact, outputs within
-    tolerance."""
-    T = 16
-    lay = gen.make_layer(gen.config(1).with_T(T), 3)
-    out, L = run_layer(lay, SCATTER, AUTO)
-    assert not L.fused_ok(T)
-    assert out["err"] == 0
-    check_routing(out, lay)
-    check_permutation_props(out, T)
-    check_output(out, lay, np.arange(T))
-
-
 @pytest.mark.parametrize("T", [1, 7])
 def test_fused_decode_hidden_1024(T):
     spec = gen.LayerSpec(T=T, H=1024, I=256, seed=12)
