@@ -346,16 +346,17 @@ def run_decode(device, steps, warmup, world, peaks):
     clocks = sampler.stop()
     ms_step = total_ms / steps
 
-    # the dominant kernels: the expert FFN of each layer, timed alone (40 per replay)
+    # the expert FFN kernel on its own (moe_expert_ffn, 40 launches per replay of its
+    # own graph): not part of the step, reported beside the step's roofline
     with torch.cuda.stream(stream):
         ffn_ms = _timed_replays(g_ffn.replay, steps, stream) / (steps * LAYERS)
     achieved = FFN_BYTES_T1 / (ffn_ms * 1e-3) / 1e9
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"],
-                "traffic": profiled_traffic("ffn_gemv", "ffn_gemv_decode_t1_ncu.txt"),
-                "kernel": "moe_expert_ffn (T=1: gate/up + SwiGLU, then down + combine-add)",
-                "algorithmic_bytes": FFN_BYTES_T1, "avg_launch_us": ffn_ms * 1e3,
-                "peak_source": peaks["source"] + " hbm_gbs"}
+    roofline_ffn = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": achieved / peaks["hbm_gbs"],
+                    "traffic": profiled_traffic("ffn_gemv", "ffn_gemv_decode_t1_ncu.txt"),
+                    "kernel": "k_ffn_gemv<false> (moe_expert_ffn at T=1: gate/up + SwiGLU, then down + combine-add)",
+                    "algorithmic_bytes": FFN_BYTES_T1, "avg_launch_us": ffn_ms * 1e3,
+                    "peak_source": peaks["source"] + " hbm_gbs"}
 
     # end to end through the public API: pinned host x -> device, 40 layers, y -> pinned host
     x_pin = torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -374,18 +375,22 @@ def run_decode(device, steps, warmup, world, peaks):
     e2e = {"value": LAYERS / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": LAYERS * H * 2,
            "d2h_bytes_per_step": LAYERS * H * 2, "ms_per_step": e2e_ms}
 
-    # the whole layer (fused decode kernel + combine): router + expert bytes per layer pass
+    # the step's dominant work, timed over the timed region above: per layer pass the fused
+    # decode kernel (route + permute + expert FFN) and its combine, router + expert bytes
     layer_bytes = LAYER_BYTES_T1
     layer_us = ms_step * 1e3 / LAYERS
-    roofline_layer = {"bound": "hbm", "achieved": layer_bytes / (layer_us * 1e-6) / 1e9, "peak": peaks["hbm_gbs"],
-                      "unit": "GB/s", "frac": layer_bytes / (layer_us * 1e-6) / 1e9 / peaks["hbm_gbs"],
-                      "kernel": "moe_decode_layer (fused route + permute + expert FFN, then combine)",
-                      "algorithmic_bytes": layer_bytes, "avg_layer_us": layer_us,
-                      "peak_source": peaks["source"] + " hbm_gbs"}
+    layer_gbs = layer_bytes / (layer_us * 1e-6) / 1e9
+    roofline = {"bound": "hbm", "achieved": layer_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": layer_gbs / peaks["hbm_gbs"],
+                "traffic": profiled_traffic("ffn_gemv", "decode_layer_fused_ncu.txt"),
+                "kernel": "moe_decode_layer: k_ffn_gemv<true> (route + permute + expert FFN) + k_combine_scatter",
+                "algorithmic_bytes": layer_bytes, "avg_layer_us": layer_us, "launches_per_layer": 2,
+                "traffic_note": "ncu DRAM bytes of the fused kernel's launch; the combine adds about 12 KB",
+                "peak_source": peaks["source"] + " hbm_gbs"}
     breakdown = _breakdown(layers, [x_dev[l:l + 1] for l in range(LAYERS)], 1, steps, stream)
     launches = _launch_count(layers[0], 1) * LAYERS
     return {"ms_per_step": ms_step, "units_per_step": LAYERS * 1, "roofline": roofline,
-            "roofline_layer": roofline_layer, "e2e": e2e,
+            "roofline_ffn": roofline_ffn, "e2e": e2e,
             "clocks": clocks, "gpu_launches": launches * steps, "breakdown_us_per_layer": breakdown,
             "_host_layers": host}
 
@@ -610,7 +615,7 @@ def decode_line(res: dict, ms: float, units: float, world: int, steps: int, warm
         "breakdown_us_per_layer": res["breakdown_us_per_layer"],
         "gpu_launches": res["gpu_launches"],
         "roofline": res["roofline"],
-        "roofline_layer": res["roofline_layer"],
+        "roofline_ffn": res["roofline_ffn"],
         "e2e": res["e2e"],
         "clocks": res["clocks"],
         "peaks": peaks,

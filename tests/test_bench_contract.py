@@ -21,7 +21,7 @@ def _fake_decode_result():
                 "traffic": 15997440}
     return {
         "ms_per_step": 0.8, "units_per_step": 40, "roofline": roofline,
-        "roofline_layer": dict(roofline, frac=0.12), "clocks": {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []},
+        "roofline_ffn": dict(roofline, frac=0.2), "clocks": {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []},
         "e2e": {"value": 47000.0, "unit": "tokens/s", "h2d_bytes_per_step": 163840, "d2h_bytes_per_step": 163840},
         "gpu_launches": 16000, "breakdown_us_per_layer": {"route": 6.0}, "_host_layers": [],
     }
