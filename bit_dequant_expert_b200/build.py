@@ -55,10 +55,17 @@ def stale() -> bool:
     return any(os.path.getmtime(p) > t for p in sources() + _deps())
 
 
+def _env() -> dict:
+    """nvcc's temporary files go to a folder inside the repository."""
+    tmpdir = os.path.join(BUILD, "tmp")
+    os.makedirs(tmpdir, exist_ok=True)
+    return dict(os.environ, TMPDIR=tmpdir)
+
+
 def _compile(src: str, extra: list[str]) -> str:
     obj = os.path.join(BUILD, os.path.basename(src) + ".o")
     cmd = [nvcc()] + NVCC_FLAGS + extra + ["-c", src, "-o", obj]
-    subprocess.check_call(cmd)
+    subprocess.check_call(cmd, env=_env())
     return obj
 
 
@@ -72,7 +79,8 @@ def build(force: bool = False, jobs: int | None = None, extra: list[str] | None 
     with cf.ThreadPoolExecutor(jobs) as ex:
         objs = list(ex.map(lambda s: _compile(s, extra), srcs))
     tmp = OUT + ".tmp.%d" % os.getpid()
-    subprocess.check_call([nvcc(), "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", tmp] + objs)
+    subprocess.check_call([nvcc(), "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", tmp] + objs,
+                          env=_env())
     os.replace(tmp, OUT)
     return OUT
 

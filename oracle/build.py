@@ -11,12 +11,19 @@ SRC = os.path.join(HERE, "moe_oracle.c")
 OUT = os.path.join(HERE, "libmoe_oracle.so")
 
 
-def build(force: bool = False, out: str = OUT, defines=()) -> str:
-    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(SRC):
+def _env() -> dict:
+    """The compiler's temporary files go to a folder inside the repository."""
+    tmpdir = os.path.join(HERE, "_build", "tmp")
+    os.makedirs(tmpdir, exist_ok=True)
+    return dict(os.environ, TMPDIR=tmpdir)
+
+
+def build(force: bool = False, out: str = OUT, defines=(), src: str = SRC) -> str:
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
         tmp = out + ".tmp.%d" % os.getpid()
         cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math"]
         cmd += ["-D%s" % d for d in defines]
-        subprocess.check_call(cmd + [SRC, "-o", tmp, "-lm"])
+        subprocess.check_call(cmd + [src, "-o", tmp, "-lm"], env=_env())
         os.replace(tmp, out)
     return out
 

@@ -11,7 +11,12 @@ if HERE not in sys.path:
     sys.path.insert(0, HERE)
 
 
+@pytest.hookimpl(tryfirst=True)
 def pytest_configure(config):
+    # temporary paths of the tests stay inside the repository (a git-ignored folder)
+    if config.option.basetemp is None:
+        os.makedirs(os.path.join(ROOT, "_build"), exist_ok=True)
+        config.option.basetemp = os.path.join(ROOT, "_build", "pytest")
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long-running CPU test")
 

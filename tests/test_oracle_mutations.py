@@ -5,11 +5,11 @@ Mutants are built from a patched copy of oracle/moe_oracle.c in a temporary
 directory; the real oracle is never touched.
 """
 import os
-import subprocess
 
 import pytest
 
 import oracle
+import oracle.build as oracle_build
 import oracle_pins
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle", "moe_oracle.c")
@@ -49,8 +49,7 @@ def test_pins_catch_mutant(name, tmp_path):
     src = tmp_path / "moe_oracle.c"
     src.write_text(text.replace(old, new))
     so = tmp_path / "libmutant.so"
-    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-ffp-contract=off",
-                           str(src), "-o", str(so), "-lm"])
+    oracle_build.build(True, out=str(so), src=str(src))   # the oracle's own compiler flags
     L = oracle.lib(str(so))
     caught = []
     for check in oracle_pins.ALL_CHECKS:
