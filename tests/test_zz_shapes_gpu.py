@@ -70,3 +70,43 @@ def test_without_shared_expert(path, mode, T):
     assert out["err"] == 0
     check_routing(out, lay)
     check_output(out, lay, np.arange(T), has_shared=False)
+
+
+def _scale_bf16(bits, e):
+    """bf16 bits times 2^e, exactly (normal inputs and results)."""
+    f = gen.bf16_to_f32(bits).astype(np.float32) * np.float32(2.0 ** e)
+    out = gen.f32_to_bf16_bits(f)
+    assert np.array_equal(gen.bf16_to_f32(out), f)
+    return out
+
+
+@pytest.mark.parametrize("path,T", [(AUTO, 8), (GEMV, 8), (AUTO, 33)])
+def test_routing_with_subnormal_logits(path, T):
+    """x and the router matrix scaled by 2^-64 each: every product and every
+    logit is subnormal in fp32.  Routing must still match the oracle bit for
+    bit, which holds only if neither side flushes subnormals to zero (a flush
+    would zero every logit and pick experts 0..7).  T = 8 covers the fused
+    decode kernel and the small router, T = 33 the tiled router."""
+    lay = dict(gen.make_layer(gen.config(0).with_T(T), 2))
+    lay["x"] = _scale_bf16(lay["x"], -64)
+    lay["w_router"] = _scale_bf16(lay["w_router"], -64)
+    logits = oracle.router_logits(lay["x"], lay["w_router"])
+    assert np.all(np.abs(logits) < 2.0 ** -126) and np.all(logits != 0)
+    out, _ = run_layer(lay, SCATTER, path)
+    assert out["err"] == 0
+    idx_ref = check_routing(out, lay)
+    assert not np.array_equal(np.sort(idx_ref, axis=1), np.tile(np.arange(8), (T, 1)))
+
+
+@pytest.mark.parametrize("path,T", [(GEMV, 8), (AUTO, 33)])
+def test_given_subnormal_logits_with_ties(path, T):
+    """Given logits that are multiples of 2^-140 (subnormal) with mass ties:
+    the top 8 by (logit desc, index asc) and their weights match the oracle."""
+    rng = np.random.default_rng(T)
+    li = (rng.integers(0, 3, size=(T, 256)) * 2.0 ** -140).astype(np.float32)
+    lay = gen.make_layer(gen.config(0).with_T(T), 2)
+    out, _ = run_layer(lay, SCATTER, path, logits_in=li)
+    assert out["err"] == 0
+    idx_ref, w_ref = oracle.select(li, 8)
+    assert np.array_equal(out["idx"], idx_ref)
+    assert np.abs(out["w"] - w_ref).max() <= 2e-6
