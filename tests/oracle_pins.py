@@ -137,6 +137,26 @@ def check_router_error_bound(L):
     assert np.array_equal(sub, gotb[[3, 1]])
 
 
+def check_router_subnormal(L):
+    """Subnormal products and partial sums are kept, not flushed to zero.
+
+    With x_h = 2^-70 (1 + (h mod 128)/128) and w_h = 2^-70 over H = 256
+    inputs, every product 2^-140 (1 + (h mod 128)/128) is an exact fp32
+    subnormal, every partial sum stays an exact multiple of 2^-149 below
+    2^-126, and the logit is sum_h of them = 383 * 2^-140 exactly; a flush of
+    subnormals to zero anywhere would give 0.
+    """
+    H, E = 256, 2
+    x = np.array([[bf16_bits(2.0 ** -70 * (1 + (h % 128) / 128)) for h in range(H)]], dtype=np.uint16)
+    wr = np.zeros((E, H), dtype=np.uint16)
+    wr[1, :] = bf16_bits(2.0 ** -70)
+    got = oracle.router_logits(x, wr, L=L)
+    want = np.float32(383 * 2.0 ** -140)
+    assert 0 < want < np.float32(2.0 ** -126)
+    assert got[0, 1] == want, (got[0, 1], want)
+    assert got[0, 0] == 0.0
+
+
 # ---------------------------------------------------------------- selection
 
 
@@ -356,6 +376,7 @@ ALL_CHECKS = [
     check_dequant_matrix_affine,
     check_router_order_golden,
     check_router_error_bound,
+    check_router_subnormal,
     check_select_example,
     check_select_bruteforce,
     check_select_ties_and_zero,

@@ -23,6 +23,10 @@ MUTANTS = {
     "group index from wrong axis": ("(n * (K / G) + k / G) * 2", "(n * (K / G) + (k / 8) % (K / G)) * 2"),
     "butterfly reversed": ("for (int off = 16; off >= 1; off /= 2)", "for (int off = 1; off <= 16; off *= 2)"),
     "chunk order reversed": ("int64_t h = 8 * c + j;", "int64_t h = 8 * c + (7 - j);"),
+    "subnormal partial sums flushed": (
+        "acc[s] = fmaf(bf16_to_float(xr[h]), bf16_to_float(wr[h]), acc[s]);",
+        "acc[s] = fmaf(bf16_to_float(xr[h]), bf16_to_float(wr[h]), acc[s]);\n"
+        "                if (fabsf(acc[s]) < 1.17549435e-38f) acc[s] = 0.0f;"),
     "router bias dropped": ("if (bias) l = l + bias[t * bias_stride + e];", "(void)bias_stride;"),
     "tie goes to higher index": ("if (best < 0 || l[e] > l[best]) best = e;",
                                  "if (best < 0 || l[e] >= l[best]) best = e;"),
