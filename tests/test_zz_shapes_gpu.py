@@ -110,3 +110,33 @@ def test_given_subnormal_logits_with_ties(path, T):
     idx_ref, w_ref = oracle.select(li, 8)
     assert np.array_equal(out["idx"], idx_ref)
     assert np.abs(out["w"] - w_ref).max() <= 2e-6
+
+
+@pytest.mark.parametrize("path,mode,T", [(AUTO, SCATTER, 8), (GEMV, SCATTER, 3), (SIMT, PAIRS, 8),
+                                         (TC, SCATTER, 33), (TC, PAIRS, 33)])
+def test_general_scale_and_bias(path, mode, T):
+    """(scale, bias) pairs of any sign and with no relation between them (the
+    synthetic layers all have positive scales and bias = -8 scale): every path
+    must compute scale * q + bias as written."""
+    rng = np.random.default_rng(100 + T)
+    lay = dict(gen.make_layer(gen.config(0).with_T(T), 4))
+    for name in ("gu_sb", "d_sb"):
+        sb = np.empty_like(lay[name])
+        sb[..., 0] = gen.f32_to_bf16_bits((0.02 * rng.standard_normal(sb.shape[:-1])).astype(np.float32))
+        sb[..., 1] = gen.f32_to_bf16_bits((0.05 * rng.standard_normal(sb.shape[:-1])).astype(np.float32))
+        lay[name] = sb
+    out, _ = run_layer(lay, mode, path)
+    assert out["err"] == 0
+    check_routing(out, lay)
+    check_output(out, lay, np.arange(T))
+
+
+@pytest.mark.parametrize("mode,T", [(SCATTER, 33), (PAIRS, 100)])
+def test_tensor_core_hidden_1024(mode, T):
+    """H = 1024, I = 256 on the tensor-core path: 16 (scale, bias) groups per
+    gate/up row and 4 per down row, four 64-column blocks of h."""
+    lay = gen.make_layer(gen.LayerSpec(T=T, H=1024, I=256, seed=12), 1)
+    out, _ = run_layer(lay, mode, TC)
+    assert out["err"] == 0
+    check_routing(out, lay)
+    check_output(out, lay, np.arange(0, T, 3))
