@@ -140,3 +140,20 @@ def test_tensor_core_hidden_1024(mode, T):
     assert out["err"] == 0
     check_routing(out, lay)
     check_output(out, lay, np.arange(0, T, 3))
+
+
+@pytest.mark.parametrize("mode", [SCATTER, PAIRS])
+def test_one_layer_across_token_counts(mode):
+    """One layer object (buffers and workspace for 64 tokens) called with
+    token counts that switch between the decode kernel, the fused decode
+    layer and the tensor-core path, as a serving loop would: the workspace's
+    arrival counter and tickets carry over from call to call, and every call
+    matches the oracle on its own tokens (a prefix of the same batch)."""
+    from bit_dequant_expert_b200.layer import MoELayer
+    lay = gen.make_layer(gen.config(0).with_T(64), 5)
+    L = MoELayer(lay, max_tokens=64, mode=mode)
+    for T in (5, 33, 1, 8, 64, 2, 8, 17):
+        out, _ = run_layer(lay, mode, AUTO, T=T, layer_obj=L)
+        assert out["err"] == 0, T
+        check_routing(out, lay, T=T)
+        check_output(out, lay, np.arange(T), T=T)
