@@ -32,6 +32,12 @@
  *    wait) set a sticky error word in the workspace and the kernels carry
  *    on with safe values; moe_get_device_error reads it.
  *  - Concurrent calls must use distinct workspaces.
+ *  - The decode kernels (moe_decode_layer, and moe_expert_ffn for T <= 8 on
+ *    the automatic or GEMV path) run one CTA per SM and wait for every CTA of
+ *    their launch.  Two of them executing at the same time on different
+ *    streams can each hold part of the SMs and starve the other; the bounded
+ *    wait then ends it with MOE_ERR_TIMEOUT.  Issue decode calls of
+ *    concurrent layers on one stream (or order their streams with events).
  *
  * Supported shapes: hidden % 256 == 0, inter % 128 == 0, num_experts == 256,
  * top_k == 8, group_size == 64, has_shared in {0, 1}, 1 <= T <= 65536.
