@@ -188,6 +188,18 @@ def barrier(world):
 # ---------------------------------------------------------- oracle timing
 
 
+def cpu_model() -> str:
+    """The host CPU's model name from /proc/cpuinfo (empty if unreadable)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return ""
+
+
 def omp_threads() -> int:
     try:
         import ctypes
@@ -250,7 +262,7 @@ def time_oracle_other_configs(budget_s: float, ids=(0, 2, 4), single_thread=(0, 
                 rate, n, dt = time_oracle_layer(lay, budget_s)
             finally:
                 _omp_set_threads(full)
-            out[str(cid)][label] = {"value": rate, "unit": UNIT, "cores": nt, "kind": "oracle",
+            out[str(cid)][label] = {"value": rate, "unit": UNIT, "cores": nt, "cpu": cpu_model(), "kind": "oracle",
                                     "sample": "first %d of %d tokens in one call, %.2f s" % (n, lay["x"].shape[0], dt)}
     return out
 
@@ -695,8 +707,6 @@ def main(argv=None):
 
     ms, units = aggregate(res["ms_per_step"], res["units_per_step"], world)
     line = decode_line(res, ms, units, world, args.steps, warmup, peaks)
-    if pre is not None:
-        line["prefill_t2048"] = pre
     if args.other_configs == "on":
         line["other_configs"] = run_other_configs(device, max(args.steps // 10, 5), warmup, peaks)
         line["small_t"] = run_other_configs(device, max(args.steps // 10, 5), warmup, peaks, small_t_specs())
@@ -704,11 +714,15 @@ def main(argv=None):
         budget = args.cpu_budget
         layers_host = res.pop("_host_layers")
         rate, n, dt = time_oracle_decode(layers_host, budget)
-        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": omp_threads(), "kind": "oracle",
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": omp_threads(), "cpu": cpu_model(),
+                                "kind": "oracle",
                                 "sample": "%d layer passes (T=1) of the first decode layers, %.1f s" % (n, dt)}
         if "other_configs" in line:
             for cid, cpu in time_oracle_other_configs(budget / 4).items():
                 line["other_configs"][cid]["cpu_baseline"] = cpu
+    if pre is not None:
+        # last key of the line, so that a reader keeping only the line's tail still sees it
+        line["prefill_t2048"] = pre
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -744,7 +758,7 @@ def run_reference(args, world, rank, warmup):
         "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic (seeded)",
         "config": {"workload": DECODE_WORKLOAD, "global_batch": 1, "seq_len": 1, "parallelism": "host cores"},
         "impl": "reference",
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": omp_threads(), "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": omp_threads(), "cpu": cpu_model(), "kind": "oracle",
                          "sample": "one layer pass (T=1) per step, layers 0-2 cycled"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }

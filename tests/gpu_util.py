@@ -62,6 +62,37 @@ def check_routing(out, lay, tokens=None, T=None):
     return idx_ref
 
 
+def check_routing_and_permutation(out, lay, T=None):
+    """Every token: indices bit-exact, weights within tolerance, and counts,
+    offsets and both row maps bit-exact against the oracle's permutation of
+    the oracle's routing."""
+    idx_ref = check_routing(out, lay, T=T)
+    counts, offsets, r2p, p2r = oracle.permute(idx_ref, 256)
+    assert np.array_equal(out["counts"], counts), "counts differ"
+    assert np.array_equal(out["offsets"], offsets), "offsets differ"
+    assert np.array_equal(out["r2p"], r2p), "row_to_pair differs"
+    assert np.array_equal(out["p2r"], p2r), "pair_to_row differs"
+    return idx_ref
+
+
+def spread_tokens(lay, n, seed):
+    """n tokens for an output check: the first and last, then as many biased
+    (hot-expert) tokens as unbiased ones when the layer has a per-token bias,
+    else a uniform draw."""
+    T = lay["x"].shape[0]
+    rng = np.random.default_rng(seed)
+    bias = lay.get("logit_bias")
+    if bias is None or not int(lay.get("bias_stride", 0)):
+        pick = rng.choice(np.arange(1, T - 1), n - 2, replace=False)
+    else:
+        biased = np.nonzero(np.asarray(bias).any(axis=1))[0]
+        plain = np.setdiff1d(np.arange(T), biased)
+        half = (n - 2) // 2
+        pick = np.concatenate([rng.choice(biased, half, replace=False),
+                               rng.choice(plain, n - 2 - half, replace=False)])
+    return np.unique(np.concatenate([[0, T - 1], pick])).astype(np.int64)
+
+
 def check_permutation_props(out, T, E=256, K=8):
     """Properties that hold at any size, on the device's own routing."""
     idx = out["idx"].reshape(T, K)
