@@ -119,7 +119,7 @@ class ClockSampler:
 
 # Kernel sources whose ncu summaries under profiles/ carry DRAM traffic per launch.
 KERNEL_SOURCES = {
-    "ffn_gemv": ["bit_dequant_expert_b200/csrc/ffn_gemv.cu"],
+    "ffn_decode": ["bit_dequant_expert_b200/csrc/ffn_decode.cu"],
     "ffn_tc": ["bit_dequant_expert_b200/csrc/ffn_tc.cu"],
 }
 KERNEL_HEADERS = ["bit_dequant_expert_b200/csrc/common.cuh", "bit_dequant_expert_b200/csrc/ptx.cuh",
@@ -365,8 +365,8 @@ def run_decode(device, steps, warmup, world, peaks):
     achieved = FFN_BYTES_T1 / (ffn_ms * 1e-3) / 1e9
     roofline_ffn = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": achieved / peaks["hbm_gbs"],
-                    "traffic": profiled_traffic("ffn_gemv", "ffn_gemv_decode_t1_ncu.txt"),
-                    "kernel": "k_ffn_gemv<false> (moe_expert_ffn at T=1: gate/up + SwiGLU, then down + combine-add)",
+                    "traffic": profiled_traffic("ffn_decode", "ffn_decode_t1_ncu.txt"),
+                    "kernel": "k_decode<false> (moe_expert_ffn at T=1: gate/up + SwiGLU, then down + vector reductions into y_acc)",
                     "algorithmic_bytes": FFN_BYTES_T1, "avg_launch_us": ffn_ms * 1e3,
                     "peak_source": peaks["source"] + " hbm_gbs"}
 
@@ -394,10 +394,10 @@ def run_decode(device, steps, warmup, world, peaks):
     layer_gbs = layer_bytes / (layer_us * 1e-6) / 1e9
     roofline = {"bound": "hbm", "achieved": layer_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": layer_gbs / peaks["hbm_gbs"],
-                "traffic": profiled_traffic("ffn_gemv", "decode_layer_fused_ncu.txt"),
-                "kernel": "moe_decode_layer: k_ffn_gemv<true> (route + permute + expert FFN) + k_combine_scatter",
+                "traffic": profiled_traffic("ffn_decode", "decode_layer_t1_ncu.txt"),
+                "kernel": "moe_decode_layer: k_decode<true> (route + permute + expert FFN) + k_combine_scatter",
                 "algorithmic_bytes": layer_bytes, "avg_layer_us": layer_us, "launches_per_layer": 2,
-                "traffic_note": "ncu DRAM bytes of the fused kernel's launch; the combine adds about 12 KB",
+                "traffic_note": "ncu DRAM bytes of the layer kernel's launch",
                 "peak_source": peaks["source"] + " hbm_gbs"}
     breakdown = _breakdown(layers, [x_dev[l:l + 1] for l in range(LAYERS)], 1, steps, stream)
     launches = _launch_count(layers[0], 1) * LAYERS
@@ -621,7 +621,7 @@ def decode_line(res: dict, ms: float, units: float, world: int, steps: int, warm
             "seq_len": 1,
             "parallelism": "replicas" if world > 1 else "single GPU",
             "l2": "inputs larger than L2 (18.2 GB of weights streamed per step; no flush)",
-            "graph": "one CUDA graph per step (40 layers x moe_decode_layer: fused route + permute + expert FFN kernel, then combine)",
+            "graph": "one CUDA graph per step (40 layers x moe_decode_layer: decode kernel + combine)",
         },
         "decode_token_per_s": world / (ms / 1e3),
         "breakdown_us_per_layer": res["breakdown_us_per_layer"],

@@ -182,8 +182,8 @@ def moe_combine(cfg, T, mode, in0, in1, pair_to_row, topk_w, y, stream=None, rai
 def moe_decode_layer(cfg, T, x, w_router, logit_bias, logit_bias_row_stride, gu_codes, gu_sb, d_codes, d_sb,
                      topk_idx, topk_w, counts, offsets, row_to_pair, pair_to_row, y_acc, y, ws, ws_bytes=None,
                      stream=None, raise_on_error=True) -> int:
-    """The whole layer for T <= 8 tokens in two launches (router, top-k and
-    permutation fused into the decode expert FFN, then the combine)."""
+    """The whole layer for T <= 8 tokens in two launches (router, top-k,
+    permutation and expert FFNs in one kernel, then the combine)."""
     n = _nbytes(ws) if ws_bytes is None else ws_bytes
     st = _lib.moe_decode_layer(ctypes.byref(cfg), T, _ptr(x), _ptr(w_router), _ptr(logit_bias),
                                logit_bias_row_stride, _ptr(gu_codes), _ptr(gu_sb), _ptr(d_codes), _ptr(d_sb),

@@ -14,12 +14,14 @@ constexpr int kWarp = 32;
 
 // Workspace header: sticky error word at byte 0, the small-T router's
 // last-block ticket at byte 4 (left at zero by every call), the decode
-// kernel's grid barrier counter at byte 8 (monotonic, 64-bit); the rest of
-// the first 256 bytes is reserved.  Scratch sections follow, 256-byte aligned.
+// kernels' launch counter at byte 8 (monotonic, 64-bit: every decode launch
+// adds its grid size, so count / grid size numbers the launches); the rest
+// of the first 256 bytes is reserved.  Scratch sections follow, 256-byte
+// aligned.
 struct WsHeader {
     int32_t error;
     uint32_t route_ticket;
-    unsigned long long grid_sync;
+    unsigned long long decode_launches;
     int32_t reserved[60];
 };
 

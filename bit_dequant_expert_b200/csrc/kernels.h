@@ -67,18 +67,28 @@ cudaError_t launch_router(const RouterArgs& a, cudaStream_t st);
 size_t permute_ws_bytes(int T, int E, int K);
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st);
 cudaError_t launch_ffn_simt(const FfnArgs& a, cudaStream_t st);
-bool ffn_gemv_supported(const FfnArgs& a);
-cudaError_t launch_ffn_gemv(const FfnArgs& a, unsigned long long* sync, cudaStream_t st);
 cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st);
 
-// Decode layer in one kernel: router logits, top-k, permutation and expert
-// FFN (scatter into y_acc); the routing outputs are written as the route and
-// permute calls would.
+// Workspace sections of the decode kernels (T <= 8): the launch counter in
+// the workspace header and the tagged router logits.
+struct DecodeWs {
+    unsigned long long* launches;
+    unsigned long long* tlogits;
+};
+size_t decode_ws_bytes(int T, int E, int I);
+DecodeWs decode_ws_carve(uint8_t* base, int T, int E, int I, unsigned long long* launches);
+
+// Expert FFNs for T <= 8 (scatter mode): one launch, y_acc overwritten.
+bool ffn_decode_supported(const FfnArgs& a);
+cudaError_t launch_ffn_decode(const FfnArgs& a, const DecodeWs& w, cudaStream_t st);
+
+// The decode layer's router logits, top-k, permutation and expert FFNs in one
+// kernel (the routing outputs written as the route and permute calls would,
+// y_acc as the FFN call would), then the combine.
 struct DecodeRoute {
     const uint16_t* w_router;
     const float* bias;
     int64_t bias_stride;
-    float* logits;
     int32_t* topk_idx;
     float* topk_w;
     int32_t* counts;
@@ -86,8 +96,8 @@ struct DecodeRoute {
     int32_t* row_to_pair;
     int32_t* pair_to_row;
 };
-bool decode_fused_supported(const FfnArgs& a);
-cudaError_t launch_decode_fused(const FfnArgs& a, const DecodeRoute& r, unsigned long long* sync, cudaStream_t st);
+bool decode_layer_supported(const FfnArgs& a);
+cudaError_t launch_decode_layer(const FfnArgs& a, const DecodeRoute& r, const DecodeWs& w, cudaStream_t st);
 bool ffn_tc_supported(const FfnArgs& a);
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st);
 

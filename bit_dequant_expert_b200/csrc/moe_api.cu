@@ -18,7 +18,7 @@ bool config_ok(const moe_config_t* c) {
 }
 
 struct WsLayout {
-    size_t logits, perm, h, xg, total;
+    size_t logits, perm, h, xg, dec, total;
 };
 
 WsLayout layout(const moe_config_t* c, int T) {
@@ -32,6 +32,8 @@ WsLayout layout(const moe_config_t* c, int T) {
     off += align256((size_t)(c->top_k + 1) * T * c->inter * sizeof(uint16_t));
     L.xg = off;
     off += align256((size_t)(c->top_k + 1) * T * c->hidden * sizeof(uint16_t));
+    L.dec = off;
+    off += decode_ws_bytes(T, c->num_experts, c->inter);
     L.total = off;
     return L;
 }
@@ -58,9 +60,14 @@ int32_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_
 // a handful of tokens, else the tensor-core kernel where its shape rules
 // hold, else the CUDA-core path.
 int32_t resolve_path(const FfnArgs& a) {
-    if (ffn_gemv_supported(a)) return MOE_PATH_GEMV;
+    if (ffn_decode_supported(a)) return MOE_PATH_GEMV;
     if (ffn_tc_supported(a)) return MOE_PATH_TC;
     return MOE_PATH_SIMT;
+}
+
+DecodeWs decode_ws(void* ws, const moe_config_t* cfg, int32_t T) {
+    return decode_ws_carve(static_cast<uint8_t*>(ws) + layout(cfg, T).dec, T, cfg->num_experts, cfg->inter,
+                           &reinterpret_cast<WsHeader*>(ws)->decode_launches);
 }
 
 FfnArgs shape_only(const moe_config_t* cfg, int32_t T) {
@@ -86,7 +93,8 @@ size_t moe_workspace_size(const moe_config_t* cfg, int32_t max_tokens) {
 
 int32_t moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
     if (!ws || ws_bytes < sizeof(WsHeader) || !aligned(ws, 256)) return MOE_ERR_WORKSPACE;
-    return cuda_status(cudaMemsetAsync(ws, 0, sizeof(WsHeader), (cudaStream_t)stream));
+    // all of it: the decode kernels' tagged words must not match a restarted launch count
+    return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream));
 }
 
 int32_t moe_route(const moe_config_t* cfg, int32_t T, const uint16_t* x, const uint16_t* w_router,
@@ -191,8 +199,8 @@ int32_t moe_expert_ffn_path(const moe_config_t* cfg, int32_t T, const uint16_t* 
             }
             return cuda_status(launch_ffn_simt(a, s));
         case MOE_PATH_GEMV:
-            if (!ffn_gemv_supported(a)) return MOE_ERR_UNSUPPORTED;
-            return cuda_status(launch_ffn_gemv(a, &reinterpret_cast<WsHeader*>(ws)->grid_sync, s));
+            if (!ffn_decode_supported(a)) return MOE_ERR_UNSUPPORTED;
+            return cuda_status(launch_ffn_decode(a, decode_ws(ws, cfg, T), s));
         case MOE_PATH_TC:
             if (!ffn_tc_supported(a)) return MOE_ERR_UNSUPPORTED;
             return cuda_status(launch_ffn_tc(a, s));
@@ -264,22 +272,18 @@ int32_t moe_decode_layer(const moe_config_t* cfg, int32_t T, const uint16_t* x, 
         return MOE_ERR_INVALID_ARG;
     FfnArgs a = shape_only(cfg, T);
     a.mode = MOE_MODE_SCATTER;
-    if (!decode_fused_supported(a)) return MOE_ERR_UNSUPPORTED;
+    if (!decode_layer_supported(a)) return MOE_ERR_UNSUPPORTED;
     a.x = x;
     a.gu_codes = gu_codes;
     a.gu_sb = gu_sb;
     a.d_codes = d_codes;
     a.d_sb = d_sb;
-    a.offsets = offsets;
-    a.row_to_pair = row_to_pair;
-    a.topk_w = topk_w;
     a.y_acc = y_acc;
     a.err = err_word(ws);
     DecodeRoute r;
     r.w_router = w_router;
     r.bias = logit_bias;
     r.bias_stride = logit_bias_row_stride;
-    r.logits = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + layout(cfg, T).logits);
     r.topk_idx = topk_idx;
     r.topk_w = topk_w;
     r.counts = counts;
@@ -287,7 +291,7 @@ int32_t moe_decode_layer(const moe_config_t* cfg, int32_t T, const uint16_t* x, 
     r.row_to_pair = row_to_pair;
     r.pair_to_row = pair_to_row;
     cudaStream_t s = (cudaStream_t)stream;
-    st = cuda_status(launch_decode_fused(a, r, &reinterpret_cast<WsHeader*>(ws)->grid_sync, s));
+    st = cuda_status(launch_decode_layer(a, r, decode_ws(ws, cfg, T), s));
     if (st) return st;
     CombineArgs c = {};
     c.T = T;
@@ -311,7 +315,7 @@ int32_t moe_launch_count(const moe_config_t* cfg, int32_t T, int32_t mode, int32
     int ffn;
     switch (path) {
         case MOE_PATH_SIMT: ffn = 2; break;
-        case MOE_PATH_GEMV: if (!ffn_gemv_supported(a)) return -1; ffn = 1; break;
+        case MOE_PATH_GEMV: if (!ffn_decode_supported(a)) return -1; ffn = 1; break;
         case MOE_PATH_TC: if (!ffn_tc_supported(a)) return -1; ffn = 3; break;
         default: return -1;
     }

@@ -24,28 +24,20 @@ __device__ __forceinline__ float key_value(uint32_t k) {
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
-// One warp per token.  Lane l holds the logits of experts l, l+32, ...; each
-// of the K rounds takes the warp-wide maximum of the value, then the lowest
-// expert index holding it, and retires the winner.  Weights are the softmax over the K selected logits, which is
-// the E-way softmax restricted to them and renormalised.  Lane r < K receives
-// the r-th expert and its weight.  A non-finite logit anywhere in the row
-// makes the selection experts 0..K-1 with weight 1/K and returns true
-// (warp-uniform).
+// One warp per token, the logits already in registers: lane l holds the
+// logits of experts l, l+32, ... in v.  Each of the K rounds takes the
+// warp-wide maximum of the value, then the lowest expert index holding it,
+// and retires the winner.  Weights are the softmax over the K selected
+// logits, which is the E-way softmax restricted to them and renormalised.
+// Lane r < K receives the r-th expert and its weight.  A non-finite logit
+// anywhere in the row makes the selection experts 0..K-1 with weight 1/K and
+// returns true (warp-uniform).
 template <int EPL, int K>
-__device__ __forceinline__ bool topk_select(int t, int E, const float* __restrict__ logits,
-                                            const float* __restrict__ bias, int64_t bias_stride, int& e_out,
-                                            float& w_out) {
+__device__ __forceinline__ bool topk_from_values(const float (&v)[EPL], int& e_out, float& w_out) {
     const int lane = threadIdx.x & 31;
-    float v[EPL];
     bool bad = false;
 #pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-        const int e = lane + 32 * i;
-        float l = __ldcg(logits + (size_t)t * E + e);
-        if (bias) l = __fadd_rn(l, bias[(int64_t)t * bias_stride + e]);
-        v[i] = l;
-        bad |= !isfinite(l);
-    }
+    for (int i = 0; i < EPL; ++i) bad |= !isfinite(v[i]);
     if (__any_sync(0xFFFFFFFFu, bad)) {
         e_out = lane;
         w_out = 1.0f / K;
@@ -95,6 +87,24 @@ __device__ __forceinline__ bool topk_select(int t, int E, const float* __restric
         }
     }
     return false;
+}
+
+// topk_from_values on token t's row of an fp32 [T, E] logits array (read
+// through L2), with an optional bias added first.
+template <int EPL, int K>
+__device__ __forceinline__ bool topk_select(int t, int E, const float* __restrict__ logits,
+                                            const float* __restrict__ bias, int64_t bias_stride, int& e_out,
+                                            float& w_out) {
+    const int lane = threadIdx.x & 31;
+    float v[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        float l = __ldcg(logits + (size_t)t * E + e);
+        if (bias) l = __fadd_rn(l, bias[(int64_t)t * bias_stride + e]);
+        v[i] = l;
+    }
+    return topk_from_values<EPL, K>(v, e_out, w_out);
 }
 
 // topk_select for token t, written to idx / wout [T, K] and counted in counts.

@@ -179,7 +179,7 @@ class MoELayer:
     def fused_ok(self, T) -> bool:
         """Whether forward() takes the two-launch decode layer for T tokens."""
         return (T <= 8 and self.mode == MOE_MODE_SCATTER and self.path == MOE_PATH_AUTO and self.E == 256
-                and self.H in (512, 1024, 2048))
+                and self.H in (512, 1024, 2048) and self.I <= 2048)
 
     def decode_fused(self, x, T, logit_bias=None, bias_stride=0, stream=None, y_out=None) -> torch.Tensor:
         """The layer for T <= 8 tokens in two launches (moe_decode_layer)."""

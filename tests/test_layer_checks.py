@@ -31,7 +31,7 @@ def _layer(calls):
     """A MoELayer with its buffers and library calls replaced by recorders."""
     L = object.__new__(MoELayer)
     L.H, L.max_tokens, L.device = H, 8, torch.device("cpu")
-    L.mode, L.path, L.E = 0, 0, 256
+    L.mode, L.path, L.E, L.I = 0, 0, 256, 512
     L.y = torch.zeros(8, H, dtype=torch.bfloat16)
     L.decode_fused = lambda x, T, *a, **k: calls.append(("fused", T)) or L.y[:T]
     L.route = lambda x, T, *a, **k: calls.append(("route", T))
