@@ -471,6 +471,51 @@ def run_prefill(device, steps, warmup, world, peaks):
             "l2": "inputs larger than L2 (455.8 MB of packed weights per layer)"}
 
 
+def run_expert_parallel(device, steps, warmup, world, rank, peaks):
+    """The expert-parallel layer (bit_dequant_expert_b200.ep): T = 2048 tokens
+    per rank, 256/N experts per rank, NCCL all-to-alls between ranks.  Timed
+    with CUDA events on the current stream around `steps` calls; each call
+    synchronises the host twice (the row counts set the exchange splits)."""
+    import torch
+    import gen
+    from bit_dequant_expert_b200 import ep
+    spec = gen.config(3)
+    T = spec.T
+    weights = gen.make_weights(spec, 0)                  # the same layer on every rank
+    x_host = gen.make_activations(spec, rank)["x"]       # each rank its own tokens
+    ops = ep.CudaEPOps(ep.shard_weights(weights, world, rank), spec.E, world, max_tokens=T, device=device)
+    del weights
+    L = ep.ExpertParallelLayer(ops, E=spec.E)
+    x = torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).to(device)
+    for _ in range(warmup):
+        L.forward(x)
+    torch.cuda.synchronize()
+    barrier(world)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        y = L.forward(x)
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    barrier(world)
+    # end to end: pinned host x in, y out, every step
+    x_pin = torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).pin_memory()
+    y_pin = torch.empty(T, spec.H, dtype=torch.bfloat16).pin_memory()
+    s.record()
+    for _ in range(steps):
+        x.copy_(x_pin, non_blocking=True)
+        y = L.forward(x)
+        y_pin.copy_(y, non_blocking=True)
+    e.record()
+    torch.cuda.synchronize()
+    e2e_ms = s.elapsed_time(e) / steps
+    errs = ops.device_errors()
+    return {"ms_per_step": ms, "e2e_ms": e2e_ms, "T": T, "device_errors": errs,
+            "recv_rows": L.last["recv"], "send_rows": L.last["send"],
+            "bytes_per_step": {"h2d": int(x_pin.numel() * 2), "d2h": int(y_pin.numel() * 2)}}
+
+
 def expert_bytes(h: int, i: int, g: int = G) -> int:
     """Packed bytes of one expert: gate/up [2i, h] and down [h, i] 4-bit codes
     plus one bf16 (scale, bias) pair per group of g inputs."""
@@ -576,17 +621,18 @@ def run_ncu_case(case, device, calls):
     import bit_dequant_expert_b200 as m
     from bit_dequant_expert_b200 import MOE_MODE_PAIRS, MOE_MODE_SCATTER
     from bit_dequant_expert_b200.layer import MoELayer, to_device
-    spec = gen.config(3 if case == "prefill-ffn" else 1)
+    prefill = case.startswith("prefill")
+    spec = gen.config(3 if prefill else 1)
     lay = gen.make_layer(spec, 0)
     T = spec.T
     L = MoELayer(lay, max_tokens=T, device=device,
-                 mode=MOE_MODE_PAIRS if case == "prefill-ffn" else MOE_MODE_SCATTER)
+                 mode=MOE_MODE_PAIRS if prefill else MOE_MODE_SCATTER)
     x = to_device(lay["x"], device)
     del lay
     L.route(x, T)
     L.permute(T)
     for _ in range(calls):
-        if case == "decode-layer":
+        if case in ("decode-layer", "prefill-layer"):
             L.forward(x)
         else:
             L.expert_ffn(x, T)
@@ -641,9 +687,12 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-prefill", action="store_true", help="skip the T=2048 prefill measurement")
+    ap.add_argument("--expert-parallel", action="store_true",
+                    help="measure the expert-parallel layer (256/N experts per rank, T=2048 per rank, all-to-all "
+                         "exchanges; its line replaces the decode line)")
     ap.add_argument("--prefill-only", action="store_true",
                     help="measure only the T=2048 prefill layer (its line replaces the decode line)")
-    ap.add_argument("--ncu-case", choices=("decode-ffn", "decode-layer", "prefill-ffn"),
+    ap.add_argument("--ncu-case", choices=("decode-ffn", "decode-layer", "prefill-ffn", "prefill-layer"),
                     help="a small case for a profiler capture: one synthetic layer, route + permute, then "
                          "--steps calls of the named kernel (decode: config 1 layer 0, T=1; prefill: "
                          "config 3, T=2048); prints the device error word and nothing timed")
@@ -676,6 +725,32 @@ def main(argv=None):
         st = run_other_configs(device, max(args.steps // 10, 5), warmup, peaks, small_t_specs())
         if rank == 0:
             print(json.dumps({"other_configs": oc, "small_t": st, "peaks": peaks}), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            barrier(world)
+            dist.destroy_process_group()
+        return 0
+
+    if args.expert_parallel:
+        r = run_expert_parallel(device, max(args.steps // 10, 5), warmup, world, rank, peaks)
+        ms, units = aggregate(r["ms_per_step"], r["T"], world)
+        e2e_ms, _ = aggregate(r["e2e_ms"], r["T"], world)
+        line = {"metric": "MoE expert-layer tokens/s (expert parallel, T=2048 per rank)",
+                "value": units / (ms / 1e3), "unit": UNIT, "n_gpus": world, "steps": max(args.steps // 10, 5),
+                "warmup": warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16 (4-bit weights, fp32 accumulation)",
+                "data": "synthetic (seeded; SplitMix64 layers shaped like the pages' model)",
+                "config": {"workload": "prefill: T=2048 per rank, uniform router, 256/N experts per rank "
+                                       "(H 2048, I 512, E 256 top-8 + shared, G 64)",
+                           "global_batch": 2048 * world, "seq_len": 2048, "parallelism": "ep%d" % world,
+                           "l2": "inputs larger than L2 (455.8 MB of packed weights per layer over all ranks)"},
+                "e2e": {"value": units / (e2e_ms / 1e3), "unit": UNIT,
+                        "h2d_bytes_per_step": r["bytes_per_step"]["h2d"],
+                        "d2h_bytes_per_step": r["bytes_per_step"]["d2h"]},
+                "rows_sent_per_rank_last_call": r["send_rows"], "device_errors": r["device_errors"],
+                "peaks": peaks}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
         if world > 1:
             import torch.distributed as dist
             barrier(world)

@@ -43,7 +43,7 @@ MOE_PATH_TC = 3
 EXPORTED = (
     "moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permute", "moe_expert_ffn",
     "moe_expert_ffn_path", "moe_combine", "moe_get_device_error", "moe_status_string", "moe_launch_count",
-    "moe_permute_static", "moe_decode_layer", "moe_wait_selftest",
+    "moe_permute_static", "moe_decode_layer", "moe_wait_selftest", "moe_gather_rows",
 )
 
 MOE_STATIC_MAX_TOKENS = 16384
@@ -77,6 +77,8 @@ _lib.moe_expert_ffn_path.argtypes = [_CFG, _I32, _P, _P, _P, _P, _P, _P, _P, _P,
                                      ctypes.c_size_t, _I32, _P]
 _lib.moe_combine.restype = _I32
 _lib.moe_combine.argtypes = [_CFG, _I32, _I32, _P, _P, _P, _P, _P, _P]
+_lib.moe_gather_rows.restype = _I32
+_lib.moe_gather_rows.argtypes = [_CFG, _I32, _P, _P, _P, _I32, _I32, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.moe_get_device_error.restype = _I32
 _lib.moe_get_device_error.argtypes = [_P, _P]
 _lib.moe_permute_static.restype = _I32
@@ -177,6 +179,14 @@ def moe_combine(cfg, T, mode, in0, in1, pair_to_row, topk_w, y, stream=None, rai
     st = _lib.moe_combine(ctypes.byref(cfg), T, mode, _ptr(in0), _ptr(in1), _ptr(pair_to_row), _ptr(topk_w), _ptr(y),
                           _stream(stream))
     return _check(st, "moe_combine", raise_on_error)
+
+
+def moe_gather_rows(cfg, T, x, row_to_pair, topk_w, row_begin, n_rows, rows_out, w_out, ws, ws_bytes=None,
+                    stream=None, raise_on_error=True) -> int:
+    st = _lib.moe_gather_rows(ctypes.byref(cfg), T, _ptr(x), _ptr(row_to_pair), _ptr(topk_w), row_begin, n_rows,
+                              _ptr(rows_out), _ptr(w_out), _ptr(ws), _nbytes(ws) if ws_bytes is None else ws_bytes,
+                              _stream(stream))
+    return _check(st, "moe_gather_rows", raise_on_error)
 
 
 def moe_decode_layer(cfg, T, x, w_router, logit_bias, logit_bias_row_stride, gu_codes, gu_sb, d_codes, d_sb,

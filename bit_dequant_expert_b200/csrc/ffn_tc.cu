@@ -618,7 +618,7 @@ bool ffn_tc_supported(const FfnArgs& a) {
     // of 128 inputs and every tile whole stages: K is 128 or a multiple of 256
     // for both GEMMs; one tile's (scale, bias) rows must fit their buffer
     auto k_ok = [](int k) { return k == 128 || (k >= 256 && k % 256 == 0); };
-    return a.E <= 256 && a.K == 8 && a.G == 64 && k_ok(a.H) && k_ok(a.I) && 128 * (a.H / 64) * 4 <= kSbBytes &&
+    return a.E <= 256 && a.K >= 1 && a.K <= 8 && a.G == 64 && k_ok(a.H) && k_ok(a.I) && 128 * (a.H / 64) * 4 <= kSbBytes &&
            128 * (a.I / 64) * 4 <= kSbBytes;
 }
 

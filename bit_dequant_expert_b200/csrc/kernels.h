@@ -63,6 +63,19 @@ struct CombineArgs {
     int32_t* err;
 };
 
+// Rows [row_begin, row_begin + n_rows) of the permutation, gathered for an
+// expert-parallel dispatch.
+struct GatherArgs {
+    int T, H, K, row_begin, n_rows;
+    const uint16_t* x;
+    const int32_t* row_to_pair;
+    const float* topk_w;
+    uint16_t* rows_out;
+    float* w_out;
+    int32_t* err;
+};
+
+cudaError_t launch_gather_dispatch(const GatherArgs& a, cudaStream_t st);
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t st);
 size_t permute_ws_bytes(int T, int E, int K);
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st);

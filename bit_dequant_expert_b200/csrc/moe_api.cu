@@ -11,11 +11,17 @@ namespace {
 
 constexpr int kMaxTokens = 65536;
 
+// Any expert count up to 256 and k up to 8: an expert-parallel rank runs the
+// expert FFN over its own shard of the experts, with each dispatched row as
+// one pair (k = 1).  The router and the permutation stay at 256 experts, top 8.
 bool config_ok(const moe_config_t* c) {
     return c && c->hidden >= 256 && c->hidden % 256 == 0 && c->hidden <= 16384 && c->inter >= 128 &&
-           c->inter % 128 == 0 && c->inter <= 8192 && c->num_experts == 256 && c->top_k == 8 &&
-           c->group_size == 64 && (c->has_shared == 0 || c->has_shared == 1);
+           c->inter % 128 == 0 && c->inter <= 8192 && c->num_experts >= 1 && c->num_experts <= 256 &&
+           c->top_k >= 1 && c->top_k <= 8 && c->top_k <= c->num_experts && c->group_size == 64 &&
+           (c->has_shared == 0 || c->has_shared == 1);
 }
+
+bool routing_shape_ok(const moe_config_t* c) { return c->num_experts == 256 && c->top_k == 8; }
 
 struct WsLayout {
     size_t logits, perm, h, xg, dec, total;
@@ -103,6 +109,7 @@ int32_t moe_route(const moe_config_t* cfg, int32_t T, const uint16_t* x, const u
     if (!ws) return MOE_ERR_WORKSPACE;
     int32_t st = check_common(cfg, T, ws, ws_bytes);
     if (st) return st;
+    if (!routing_shape_ok(cfg)) return MOE_ERR_UNSUPPORTED;
     if (!topk_idx || !topk_w || !counts) return MOE_ERR_INVALID_ARG;
     if (!logits_in && (!x || !w_router)) return MOE_ERR_INVALID_ARG;
     if (logit_bias_row_stride < 0) return MOE_ERR_INVALID_ARG;
@@ -133,6 +140,7 @@ int32_t moe_permute(const moe_config_t* cfg, int32_t T, const int32_t* topk_idx,
     if (!ws) return MOE_ERR_WORKSPACE;
     int32_t st = check_common(cfg, T, ws, ws_bytes);
     if (st) return st;
+    if (!routing_shape_ok(cfg)) return MOE_ERR_UNSUPPORTED;
     if (!topk_idx || !offsets || !row_to_pair || !pair_to_row) return MOE_ERR_INVALID_ARG;
     if (!aligned(topk_idx, 4) || !aligned(counts, 4) || !aligned(offsets, 4) || !aligned(row_to_pair, 4) ||
         !aligned(pair_to_row, 4))
@@ -225,6 +233,7 @@ int32_t moe_combine(const moe_config_t* cfg, int32_t T, int32_t mode, const void
     if (!in0 || !y) return MOE_ERR_INVALID_ARG;
     if (mode == MOE_MODE_PAIRS && (!pair_to_row || !topk_w || (cfg->has_shared && !in1)))
         return MOE_ERR_INVALID_ARG;
+    if (mode == MOE_MODE_PAIRS && cfg->top_k != 8) return MOE_ERR_UNSUPPORTED;
     if (!aligned(in0, 16) || !aligned(in1, 16) || !aligned(y, 16) || !aligned(pair_to_row, 4) ||
         !aligned(topk_w, 4))
         return MOE_ERR_INVALID_ARG;
@@ -241,6 +250,34 @@ int32_t moe_combine(const moe_config_t* cfg, int32_t T, int32_t mode, const void
     a.y = y;
     a.err = nullptr;   // no workspace here: out-of-range rows are clamped, the permute already reported them
     return cuda_status(launch_combine(a, (cudaStream_t)stream));
+}
+
+int32_t moe_gather_rows(const moe_config_t* cfg, int32_t T, const uint16_t* x, const int32_t* row_to_pair,
+                        const float* topk_w, int32_t row_begin, int32_t n_rows, uint16_t* rows_out, float* w_out,
+                        void* ws, size_t ws_bytes, void* stream) {
+    if (!ws) return MOE_ERR_WORKSPACE;
+    int32_t st = check_common(cfg, T, ws, ws_bytes);
+    if (st) return st;
+    if (row_begin < 0 || n_rows < 0 || (int64_t)row_begin + n_rows > (int64_t)T * cfg->top_k)
+        return MOE_ERR_INVALID_ARG;
+    if (n_rows == 0) return MOE_OK;
+    if (!x || !row_to_pair || !rows_out) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(rows_out, 16) || !aligned(row_to_pair, 4) || !aligned(topk_w, 4) ||
+        !aligned(w_out, 4))
+        return MOE_ERR_INVALID_ARG;
+    GatherArgs a;
+    a.T = T;
+    a.H = cfg->hidden;
+    a.K = cfg->top_k;
+    a.row_begin = row_begin;
+    a.n_rows = n_rows;
+    a.x = x;
+    a.row_to_pair = row_to_pair;
+    a.topk_w = topk_w;
+    a.rows_out = rows_out;
+    a.w_out = w_out;
+    a.err = err_word(ws);
+    return cuda_status(launch_gather_dispatch(a, (cudaStream_t)stream));
 }
 
 int32_t moe_get_device_error(const void* ws, void* stream) {
@@ -261,6 +298,7 @@ int32_t moe_decode_layer(const moe_config_t* cfg, int32_t T, const uint16_t* x, 
     if (!ws) return MOE_ERR_WORKSPACE;
     int32_t st = check_common(cfg, T, ws, ws_bytes);
     if (st) return st;
+    if (!routing_shape_ok(cfg)) return MOE_ERR_UNSUPPORTED;
     if (!x || !w_router || !gu_codes || !gu_sb || !d_codes || !d_sb || !topk_idx || !topk_w || !counts ||
         !offsets || !row_to_pair || !pair_to_row || !y_acc || !y)
         return MOE_ERR_INVALID_ARG;

@@ -33,15 +33,19 @@
  *    on with safe values; moe_get_device_error reads it.
  *  - Concurrent calls must use distinct workspaces.
  *  - The decode kernels (moe_decode_layer, and moe_expert_ffn for T <= 8 on
- *    the automatic or GEMV path) run one CTA per SM and wait for every CTA of
- *    their launch.  Two of them executing at the same time on different
- *    streams can each hold part of the SMs and starve the other; the bounded
- *    wait then ends it with MOE_ERR_TIMEOUT.  Issue decode calls of
- *    concurrent layers on one stream (or order their streams with events).
+ *    the automatic or GEMV path) run one CTA per SM, read words that other
+ *    CTAs of the same launch write, and are launched as cooperative grids:
+ *    the launch fails (MOE_ERR_CUDA) rather than starting when the CTAs
+ *    cannot all be resident.  Issue decode calls of concurrent layers on
+ *    one stream (or order their streams with events).
  *
- * Supported shapes: hidden % 256 == 0, inter % 128 == 0, num_experts == 256,
- * top_k == 8, group_size == 64, has_shared in {0, 1}, 1 <= T <= 65536.
- * Anything else returns MOE_ERR_UNSUPPORTED.
+ * Supported shapes: hidden % 256 == 0, inter % 128 == 0, group_size == 64,
+ * has_shared in {0, 1}, 1 <= T <= 65536.  The router, the permutation and
+ * moe_decode_layer need num_experts == 256 and top_k == 8.  moe_expert_ffn,
+ * moe_gather_rows and the scatter combine also take any 1 <= num_experts <=
+ * 256 and 1 <= top_k <= min(8, num_experts): an expert-parallel rank runs
+ * its shard of the experts over dispatched rows with top_k == 1.  Anything
+ * else returns MOE_ERR_UNSUPPORTED.
  *
  * Packed weights of an [N, K] matrix (N outputs, K inputs), matrices of all
  * experts stacked, shared expert last (index num_experts):
@@ -97,7 +101,8 @@ typedef struct {
  * and zero-fills it once, or calls moe_workspace_init. */
 size_t moe_workspace_size(const moe_config_t* cfg, int32_t max_tokens);
 
-/* Clears the workspace's sticky error word (async on stream). */
+/* Zero-fills all ws_bytes of the workspace (async on stream): the sticky
+ * error word, the decode kernels' launch counter and their tagged words. */
 int32_t moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
 
 /*
@@ -192,9 +197,11 @@ int32_t moe_combine(const moe_config_t* cfg, int32_t T, int32_t mode, const void
  * Lily pages: "Perplexity built an inference engine for one model, one
  * chip", third paragraph (the routing decision stays on the GPU with the
  * expert work; the decode step as few kernels as possible).
- * The first kernel computes the router logits over all CTAs, meets at a
- * grid-wide (bounded) barrier, selects the top-k and builds the permutation
- * in every CTA, then runs the decode expert FFN; the second converts y_acc.
+ * The first kernel computes the router logits over all CTAs and publishes
+ * each tagged with the launch's number; every CTA polls (bounded) until it
+ * holds all of a token's logits, selects the top-k, builds the list of
+ * active experts and runs its share of the decode expert FFN, and the last
+ * CTA writes the routing outputs; the second kernel converts y_acc.
  * Supported: 1 <= T <= 8, hidden 512, 1024 or 2048, E == 256, k == 8;
  * otherwise MOE_ERR_UNSUPPORTED before any launch (use the four calls).
  * Same pointer rules as the four calls; the workspace must hold T tokens.
@@ -205,6 +212,26 @@ int32_t moe_decode_layer(const moe_config_t* cfg, int32_t T, const uint16_t* x, 
                          float* topk_w, int32_t* counts, int32_t* offsets, int32_t* row_to_pair,
                          int32_t* pair_to_row, float* y_acc, uint16_t* y, void* ws, size_t ws_bytes,
                          void* stream);
+
+/*
+ * moe_gather_rows: the dispatch step of expert parallelism.  A rank holding
+ * the experts [e0, e1) receives from every rank the permuted rows
+ * offsets[e0] .. offsets[e1]-1 of that rank's permutation; this call copies
+ * such a block out of the activations, in row order.
+ *   x            bf16 [T, H] activations; row_to_pair int32 [T*k] from
+ *                moe_permute; topk_w nullable fp32 [T*k] from moe_route.
+ *   row_begin, n_rows  the block [row_begin, row_begin + n_rows) of rows,
+ *                inside [0, T*k) (else MOE_ERR_INVALID_ARG); n_rows 0 does
+ *                nothing.
+ *   rows_out     bf16 [n_rows, H]: rows_out[i] = x[row_to_pair[row_begin+i] / k].
+ *   w_out        nullable fp32 [n_rows]: w_out[i] = topk_w[row_to_pair[row_begin+i]]
+ *                (0 when topk_w is NULL).
+ * A pair index outside [0, T*k) zero-fills its row and sets MOE_ERR_BOUNDS.
+ * The workspace is only read for its error word (size checked for T).
+ */
+int32_t moe_gather_rows(const moe_config_t* cfg, int32_t T, const uint16_t* x, const int32_t* row_to_pair,
+                        const float* topk_w, int32_t row_begin, int32_t n_rows, uint16_t* rows_out, float* w_out,
+                        void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronises `stream` and returns the workspace's sticky device error
  * (MOE_OK if none), or MOE_ERR_CUDA if the synchronisation failed. */

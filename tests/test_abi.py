@@ -37,9 +37,13 @@ def test_workspace_size_and_config_checks():
     assert 0 < n1 < n2 and n1 % 256 == 0 and n2 % 256 == 0
     # (k+1) T I bf16 rows of h, T E fp32 logits at least
     assert n2 >= 9 * 2048 * 512 * 2 + 2048 * 256 * 4
-    for bad in (m.config(hidden=300), m.config(inter=100), m.config(num_experts=128), m.config(top_k=4),
+    for bad in (m.config(hidden=300), m.config(inter=100), m.config(num_experts=0), m.config(num_experts=257),
+                m.config(top_k=0), m.config(top_k=9), m.config(num_experts=4, top_k=8),
                 m.config(group_size=32), m.config(has_shared=2)):
         assert m.moe_workspace_size(bad, 16) == 0
+    # an expert-parallel shard: fewer experts, one pair per row
+    assert m.moe_workspace_size(m.config(num_experts=128, top_k=1, has_shared=0), 4096) > 0
+    assert m.moe_workspace_size(m.config(num_experts=32, top_k=4), 16) > 0
     assert m.moe_workspace_size(cfg, 0) == 0
     assert m.moe_workspace_size(cfg, 65537) == 0
 
@@ -79,6 +83,39 @@ def test_host_validation_before_launch():
     assert st == m.MOE_ERR_INVALID_ARG
     assert m.moe_get_device_error(None, 0) == m.MOE_ERR_WORKSPACE
     assert m.moe_status_string(m.MOE_ERR_NONFINITE) == "MOE_ERR_NONFINITE"
+
+
+def test_expert_shard_validation_before_launch():
+    """An expert shard (fewer experts, top_k 1) may run the expert FFN, the
+    row gather and the scatter combine; the router, the permutation, the pairs
+    combine and the fused decode layer stay at 256 experts, top 8."""
+    import bit_dequant_expert_b200 as m
+    sh = m.config(num_experts=128, top_k=1, has_shared=0)
+    need = m.moe_workspace_size(sh, 64)
+    assert _route(sh, 64, need) == m.MOE_ERR_UNSUPPORTED
+    st = m.moe_permute(sh, 64, FAKE, None, FAKE, FAKE, FAKE, FAKE, ws_bytes=need, stream=0, raise_on_error=False)
+    assert st == m.MOE_ERR_UNSUPPORTED
+    assert _decode(m.config(num_experts=128), 1, m.moe_workspace_size(m.config(num_experts=128), 1)) == \
+        m.MOE_ERR_UNSUPPORTED
+    st = m.moe_combine(sh, 64, m.MOE_MODE_PAIRS, FAKE, None, FAKE, FAKE, FAKE, stream=0, raise_on_error=False)
+    assert st == m.MOE_ERR_UNSUPPORTED
+    # the row gather: the block must lie inside [0, T*k), the pointers be set and aligned
+    cfg = m.config()
+    full = m.moe_workspace_size(cfg, 64)
+
+    def gather(T=64, begin=0, n=8, x=FAKE, rows=FAKE, w=None, ws=FAKE, nbytes=full):
+        return m.moe_gather_rows(cfg, T, x, FAKE, None, begin, n, rows, w, ws, ws_bytes=nbytes, stream=0,
+                                 raise_on_error=False)
+
+    assert gather(begin=-1) == m.MOE_ERR_INVALID_ARG
+    assert gather(begin=500, n=13) == m.MOE_ERR_INVALID_ARG
+    assert gather(n=-1) == m.MOE_ERR_INVALID_ARG
+    assert gather(n=0, x=None, rows=None) == m.MOE_OK       # nothing to copy, nothing launched
+    assert gather(x=None) == m.MOE_ERR_INVALID_ARG
+    assert gather(rows=FAKE + 8) == m.MOE_ERR_INVALID_ARG
+    assert gather(w=FAKE + 2) == m.MOE_ERR_INVALID_ARG
+    assert gather(ws=None) == m.MOE_ERR_WORKSPACE
+    assert gather(nbytes=256) == m.MOE_ERR_WORKSPACE
 
 
 def _decode(cfg, T, ws_bytes, x=FAKE, y=FAKE, bias=None, stride=0):
