@@ -46,6 +46,10 @@ def lib():
                                         ctypes.c_int64]
         _lib.gen_partial_shuffle.argtypes = [ctypes.c_uint64, ctypes.c_int32, ctypes.c_int32,
                                              ctypes.c_void_p, ctypes.c_void_p]
+        _lib.gen_uniform_f32.argtypes = [ctypes.c_uint64, ctypes.c_double, ctypes.c_double, ctypes.c_void_p,
+                                         ctypes.c_int64]
+        _lib.gen_normal_f32.argtypes = [ctypes.c_uint64, ctypes.c_double, ctypes.c_void_p, ctypes.c_int64]
+        _lib.gen_unit_bf16.argtypes = [ctypes.c_uint64, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p]
     return _lib
 
 
@@ -166,3 +170,76 @@ def f32_to_bf16_bits(f: np.ndarray) -> np.ndarray:
     u = np.ascontiguousarray(f, dtype=np.float32).view(np.uint32).astype(np.uint64)
     u = u + 0x7FFF + ((u >> 16) & 1)
     return (u >> 16).astype(np.uint16)
+
+
+# ---------------------------------------------------------------- recurrent-state scan inputs
+
+TID_GDN_Q, TID_GDN_K, TID_GDN_V, TID_GDN_G, TID_GDN_BETA, TID_GDN_S0 = range(20, 26)
+
+
+@dataclasses.dataclass(frozen=True)
+class ScanSpec:
+    """Shape and seed of one synthetic Gated DeltaNet scan: B sequences of T
+    new tokens, Hk key heads and Hv value heads (Hv a multiple of Hk) of dk
+    and dv channels, 30 layers in a decode step."""
+    B: int
+    T: int
+    Hk: int = 16
+    Hv: int = 32
+    dk: int = 128
+    dv: int = 128
+    seed: int = 0
+    layers: int = 1
+    name: str = ""
+
+    def with_T(self, T: int) -> "ScanSpec":
+        return dataclasses.replace(self, T=T)
+
+    def with_B(self, B: int) -> "ScanSpec":
+        return dataclasses.replace(self, B=B)
+
+
+SCAN_CONFIGS = {
+    0: ScanSpec(B=2, T=17, Hk=2, Hv=4, seed=10, name="tiny B=2 T=17 Hk=2 Hv=4"),
+    1: ScanSpec(B=8, T=1, seed=11, layers=30, name="decode B=8 T=1 x30 layers"),
+    2: ScanSpec(B=1, T=4, seed=12, layers=30, name="verification B=1 T=4 x30 layers"),
+    3: ScanSpec(B=1, T=2048, seed=13, name="prefill B=1 T=2048"),
+}
+
+
+def scan_config(i: int) -> ScanSpec:
+    return SCAN_CONFIGS[i]
+
+
+def uniform_f32(key: int, lo: float, hi: float, n: int) -> np.ndarray:
+    out = np.empty(n, dtype=np.float32)
+    lib().gen_uniform_f32(key, lo, hi, _ptr(out), n)
+    return out
+
+
+def normal_f32(key: int, std: float, n: int) -> np.ndarray:
+    out = np.empty(n, dtype=np.float32)
+    lib().gen_normal_f32(key, std, _ptr(out), n)
+    return out
+
+
+def unit_bf16(key: int, nvec: int, dim: int) -> np.ndarray:
+    out = np.empty(nvec * dim, dtype=np.uint16)
+    lib().gen_unit_bf16(key, nvec, dim, _ptr(out))
+    return out.reshape(nvec, dim)
+
+
+def make_scan(spec: ScanSpec, layer: int = 0) -> dict:
+    """Inputs of one scan: q, k unit vectors (bf16 [B,T,Hk,dk]), v ~ N(0,1)
+    (bf16 [B,T,Hv,dv]), g (the log of the decay) uniform in [log 0.9, 0) so
+    that the decay lies in [0.9, 1) (fp32 [B,T,Hv]), beta uniform in
+    [0.05, 0.95) (fp32 [B,T,Hv]), initial state ~ N(0, 0.1) (fp32
+    [B,Hv,dv,dk]), and the output scale dk^-1/2."""
+    B, T, Hk, Hv, dk, dv, s = spec.B, spec.T, spec.Hk, spec.Hv, spec.dk, spec.dv, spec.seed
+    q = unit_bf16(key(s, TID_GDN_Q, layer), B * T * Hk, dk).reshape(B, T, Hk, dk)
+    k = unit_bf16(key(s, TID_GDN_K, layer), B * T * Hk, dk).reshape(B, T, Hk, dk)
+    v = normal_bf16(key(s, TID_GDN_V, layer), 1.0, B * T * Hv * dv).reshape(B, T, Hv, dv)
+    g = uniform_f32(key(s, TID_GDN_G, layer), -0.10536051565782628, 0.0, B * T * Hv).reshape(B, T, Hv)
+    beta = uniform_f32(key(s, TID_GDN_BETA, layer), 0.05, 0.95, B * T * Hv).reshape(B, T, Hv)
+    S0 = normal_f32(key(s, TID_GDN_S0, layer), 0.1, B * Hv * dv * dk).reshape(B, Hv, dv, dk)
+    return dict(q=q, k=k, v=v, g=g, beta=beta, S0=S0, scale=float(dk) ** -0.5)

@@ -106,3 +106,36 @@ void gen_partial_shuffle(uint64_t key, int32_t n, int32_t m, int32_t* out_first_
         out_first_m[j] = scratch_n[j];
     }
 }
+
+/* ---- inputs of the recurrent-state scan (a second workload of the pages) */
+
+/* out[i] = float(lo + (hi - lo) * u), u = the top 24 bits of draw i / 2^24 in [0, 1). */
+void gen_uniform_f32(uint64_t key, double lo, double hi, float* out, int64_t n) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        double u = (double)(gen_draw(key, (uint64_t)i) >> 40) * 0x1.0p-24;
+        out[i] = (float)(lo + (hi - lo) * u);
+    }
+}
+
+/* out[i] = float(std * N(0,1)). */
+void gen_normal_f32(uint64_t key, double std, float* out, int64_t n) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) out[i] = (float)(std * normal_at(key, i));
+}
+
+/* nvec vectors of dim elements drawn uniformly on the unit sphere: N(0,1)
+ * elements (element j of vector v is normal j + v*dim of the stream) divided
+ * by their Euclidean norm in double, then rounded to fp32 and to bf16. */
+void gen_unit_bf16(uint64_t key, int64_t nvec, int64_t dim, uint16_t* out) {
+#pragma omp parallel for schedule(static)
+    for (int64_t v = 0; v < nvec; ++v) {
+        double ss = 0.0;
+        for (int64_t j = 0; j < dim; ++j) {
+            double z = normal_at(key, v * dim + j);
+            ss += z * z;
+        }
+        double inv = ss > 0.0 ? 1.0 / sqrt(ss) : 0.0;
+        for (int64_t j = 0; j < dim; ++j) out[v * dim + j] = f32_to_bf16((float)(normal_at(key, v * dim + j) * inv));
+    }
+}

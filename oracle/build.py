@@ -9,6 +9,8 @@ import subprocess
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "moe_oracle.c")
 OUT = os.path.join(HERE, "libmoe_oracle.so")
+GDN_SRC = os.path.join(HERE, "gdn_oracle.c")
+GDN_OUT = os.path.join(HERE, "libgdn_oracle.so")
 
 
 def _env() -> dict:
@@ -32,5 +34,15 @@ def ensure_built() -> str:
     return build(False)
 
 
+def build_gdn(force: bool = False, out: str = GDN_OUT, src: str = GDN_SRC) -> str:
+    """The recurrent-scan oracle (a separate library, same compiler flags)."""
+    return build(force, out=out, src=src)
+
+
+def ensure_gdn_built() -> str:
+    return build_gdn(False)
+
+
 if __name__ == "__main__":
     print(build(True))
+    print(build_gdn(True))
