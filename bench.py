@@ -516,6 +516,85 @@ def run_expert_parallel(device, steps, warmup, world, rank, peaks):
             "bytes_per_step": {"h2d": int(x_pin.numel() * 2), "d2h": int(y_pin.numel() * 2)}}
 
 
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # 148 SMs x 128 fp32 lanes x fma x clocks.max.sm
+
+
+def run_gdn(device, steps, warmup, peaks):
+    """The Gated DeltaNet scan (gdn_scan, one launch per layer): decode
+    (8 sequences x 1 token) and verification (1 sequence x 4 tokens) steps
+    over 30 layers with a state each, updated in place step after step, and
+    a 2048-token prefill of one layer.  CUDA graph of a step, CUDA events on
+    its stream."""
+    import torch
+    import gen
+    import bit_dequant_expert_b200 as m
+
+    def dev(a):
+        a = np.ascontiguousarray(a)
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+        return torch.from_numpy(a).to(device)
+
+    out = {}
+    flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    for name, ci in (("decode", 1), ("verify", 2), ("prefill", 3)):
+        spec = gen.scan_config(ci)
+        B, T, Hk, Hv, dk, dv = spec.B, spec.T, spec.Hk, spec.Hv, spec.dk, spec.dv
+        layers = []
+        for l in range(spec.layers):
+            d = gen.make_scan(spec, l)
+            t = {n: dev(d[n]) for n in ("q", "k", "v", "g", "beta", "S0")}
+            t["o"] = torch.empty(B, T, Hv, dv, dtype=torch.bfloat16, device=device)
+            t["scale"] = d["scale"]
+            layers.append(t)
+        stream = torch.cuda.Stream(device=device)
+
+        def step():
+            for t in layers:
+                m.gdn_scan(B, T, Hk, Hv, dk, dv, t["q"], t["k"], t["v"], t["g"], t["beta"], t["scale"], t["S0"],
+                           t["S0"], t["o"])
+
+        with torch.cuda.stream(stream):
+            step()
+        torch.cuda.synchronize()
+        g = _capture(step, stream)
+        state_bytes = B * Hv * dv * dk * 4
+        io_bytes = 2 * B * T * Hk * dk * 2 + 2 * B * T * Hv * dv * 2 + 2 * B * T * Hv * 4
+        per_layer = 2 * state_bytes + io_bytes
+        resident = spec.layers * state_bytes
+        with torch.cuda.stream(stream):
+            for _ in range(warmup):
+                g.replay()
+            n = max(steps, 3)
+            if resident < 2 * 126 * 2 ** 20:
+                ms = _timed_flushed(g.replay, n, stream, lambda: flush_buf.zero_()) / n
+                l2 = "L2 flushed between timed steps (256 MB write outside the events)"
+            else:
+                ms = _timed_replays(g.replay, n, stream) / n
+                l2 = "inputs larger than L2 (%.0f MB of state per step)" % (resident / 2 ** 20)
+        us_layer = ms * 1e3 / spec.layers
+        gbs = per_layer / (us_layer * 1e-6) / 1e9
+        flops = 7.0 * B * T * Hv * dv * dk
+        tflops = flops / (us_layer * 1e-6) / 1e12
+        r = {"workload": "%s: B=%d sequences x T=%d tokens, Hk %d, Hv %d, dk %d, dv %d, %d layer%s" %
+                         (name, B, T, Hk, Hv, dk, dv, spec.layers, "s" if spec.layers > 1 else ""),
+             "tokens_per_s": B * T / (ms * 1e-3), "ms_per_step": ms, "us_per_layer": us_layer,
+             "gpu_launches_per_step": spec.layers, "l2": l2,
+             "algorithmic_bytes_per_layer": per_layer, "algorithmic_flops_per_layer": flops}
+        if name == "prefill":
+            r["roofline"] = {"bound": "alu", "achieved": tflops, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
+                             "frac": tflops / FP32_PEAK_TFLOPS,
+                             "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1.965 GHz",
+                             "note": "one token after another: 2048 dependent steps per state row"}
+        else:
+            r["roofline"] = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": gbs / peaks["hbm_gbs"], "peak_source": peaks["source"] + " hbm_gbs"}
+        out[name] = r
+        del layers, g
+        torch.cuda.synchronize()
+    return out
+
+
 def expert_bytes(h: int, i: int, g: int = G) -> int:
     """Packed bytes of one expert: gate/up [2i, h] and down [h, i] 4-bit codes
     plus one bf16 (scale, bias) pair per group of g inputs."""
@@ -618,6 +697,22 @@ def run_ncu_case(case, device, calls):
     """One layer for a profiler: route + permute, then `calls` launches of the kernel under study."""
     import torch
     import gen
+    if case.startswith("gdn"):
+        import bit_dequant_expert_b200 as m
+        spec = gen.scan_config(1 if case == "gdn-decode" else 3)
+        d = gen.make_scan(spec, 0)
+        t = {}
+        for n in ("q", "k", "v", "g", "beta", "S0"):
+            a = np.ascontiguousarray(d[n])
+            t[n] = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16
+                    else torch.from_numpy(a)).to(device)
+        o = torch.empty(spec.B, spec.T, spec.Hv, spec.dv, dtype=torch.bfloat16, device=device)
+        for _ in range(calls):
+            m.gdn_scan(spec.B, spec.T, spec.Hk, spec.Hv, spec.dk, spec.dv, t["q"], t["k"], t["v"], t["g"],
+                       t["beta"], d["scale"], t["S0"], t["S0"], o)
+        torch.cuda.synchronize()
+        print(json.dumps({"ncu_case": case, "calls": calls}))
+        return 0
     import bit_dequant_expert_b200 as m
     from bit_dequant_expert_b200 import MOE_MODE_PAIRS, MOE_MODE_SCATTER
     from bit_dequant_expert_b200.layer import MoELayer, to_device
@@ -687,12 +782,14 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-prefill", action="store_true", help="skip the T=2048 prefill measurement")
+    ap.add_argument("--no-gdn", action="store_true", help="skip the Gated DeltaNet scan measurement")
     ap.add_argument("--expert-parallel", action="store_true",
                     help="measure the expert-parallel layer (256/N experts per rank, T=2048 per rank, all-to-all "
                          "exchanges; its line replaces the decode line)")
     ap.add_argument("--prefill-only", action="store_true",
                     help="measure only the T=2048 prefill layer (its line replaces the decode line)")
-    ap.add_argument("--ncu-case", choices=("decode-ffn", "decode-layer", "prefill-ffn", "prefill-layer"),
+    ap.add_argument("--ncu-case", choices=("decode-ffn", "decode-layer", "prefill-ffn", "prefill-layer", "gdn-decode",
+                                                   "gdn-prefill"),
                     help="a small case for a profiler capture: one synthetic layer, route + permute, then "
                          "--steps calls of the named kernel (decode: config 1 layer 0, T=1; prefill: "
                          "config 3, T=2048); prints the device error word and nothing timed")
@@ -795,6 +892,8 @@ def main(argv=None):
         if "other_configs" in line:
             for cid, cpu in time_oracle_other_configs(budget / 4).items():
                 line["other_configs"][cid]["cpu_baseline"] = cpu
+    if not args.no_gdn:
+        line["gdn_scan"] = run_gdn(device, max(args.steps // 10, 5), warmup, peaks)
     if pre is not None:
         # last key of the line, so that a reader keeping only the line's tail still sees it
         line["prefill_t2048"] = pre

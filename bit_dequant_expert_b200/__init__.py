@@ -43,7 +43,7 @@ MOE_PATH_TC = 3
 EXPORTED = (
     "moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permute", "moe_expert_ffn",
     "moe_expert_ffn_path", "moe_combine", "moe_get_device_error", "moe_status_string", "moe_launch_count",
-    "moe_permute_static", "moe_decode_layer", "moe_wait_selftest", "moe_gather_rows",
+    "moe_permute_static", "moe_decode_layer", "moe_wait_selftest", "moe_gather_rows", "gdn_scan",
 )
 
 MOE_STATIC_MAX_TOKENS = 16384
@@ -77,6 +77,8 @@ _lib.moe_expert_ffn_path.argtypes = [_CFG, _I32, _P, _P, _P, _P, _P, _P, _P, _P,
                                      ctypes.c_size_t, _I32, _P]
 _lib.moe_combine.restype = _I32
 _lib.moe_combine.argtypes = [_CFG, _I32, _I32, _P, _P, _P, _P, _P, _P]
+_lib.gdn_scan.restype = _I32
+_lib.gdn_scan.argtypes = [_I32] * 6 + [_P] * 5 + [ctypes.c_float, _P, _P, _P, _P]
 _lib.moe_gather_rows.restype = _I32
 _lib.moe_gather_rows.argtypes = [_CFG, _I32, _P, _P, _P, _I32, _I32, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.moe_get_device_error.restype = _I32
@@ -187,6 +189,14 @@ def moe_gather_rows(cfg, T, x, row_to_pair, topk_w, row_begin, n_rows, rows_out,
                               _ptr(rows_out), _ptr(w_out), _ptr(ws), _nbytes(ws) if ws_bytes is None else ws_bytes,
                               _stream(stream))
     return _check(st, "moe_gather_rows", raise_on_error)
+
+
+def gdn_scan(B, T, Hk, Hv, dk, dv, q, k, v, g, beta, scale, state_in, state_out, o, stream=None,
+             raise_on_error=True) -> int:
+    """Gated DeltaNet recurrent scan (include/gdn_b200.h)."""
+    st = _lib.gdn_scan(B, T, Hk, Hv, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
+                       _ptr(state_in), _ptr(state_out), _ptr(o), _stream(stream))
+    return _check(st, "gdn_scan", raise_on_error)
 
 
 def moe_decode_layer(cfg, T, x, w_router, logit_bias, logit_bias_row_stride, gu_codes, gu_sb, d_codes, d_sb,

@@ -76,6 +76,23 @@ struct GatherArgs {
 };
 
 cudaError_t launch_gather_dispatch(const GatherArgs& a, cudaStream_t st);
+
+// Gated DeltaNet recurrent scan (gdn_scan in the C ABI).
+struct GdnArgs {
+    int B, T, Hk, Hv, dk, dv;
+    const uint16_t* q;        // [B, T, Hk, dk] bf16
+    const uint16_t* k;        // [B, T, Hk, dk] bf16
+    const uint16_t* v;        // [B, T, Hv, dv] bf16
+    const float* g;           // [B, T, Hv] log of the decay
+    const float* beta;        // [B, T, Hv]
+    float scale;
+    const float* state_in;    // [B, Hv, dv, dk]
+    float* state_out;         // [B, Hv, dv, dk] (may equal state_in)
+    uint16_t* o;              // [B, T, Hv, dv] bf16
+};
+
+bool gdn_scan_supported(const GdnArgs& a);
+cudaError_t launch_gdn_scan(const GdnArgs& a, cudaStream_t st);
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t st);
 size_t permute_ws_bytes(int T, int E, int K);
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st);

@@ -6,19 +6,21 @@ import re
 
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "moe_b200.h")
+HEADERS = [os.path.join(ROOT, "include", h) for h in ("moe_b200.h", "gdn_b200.h")]
 
 
 def declared_functions():
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(moe_\w+)\s*\(", text, flags=re.M)))
+    names = set()
+    for header in HEADERS:
+        text = re.sub(r"/\*.*?\*/", "", open(header).read(), flags=re.S)
+        names |= set(re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b((?:moe|gdn)_\w+)\s*\(", text, flags=re.M))
+    return sorted(names)
 
 
 def test_header_declares_the_layer_calls():
     names = declared_functions()
     for n in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_workspace_size",
-              "moe_get_device_error"):
+              "moe_get_device_error", "moe_gather_rows", "gdn_scan"):
         assert n in names
 
 
@@ -176,3 +178,24 @@ def test_launch_count_per_path():
     assert m.moe_launch_count(cfg, 2048, SC, m.MOE_PATH_GEMV) == -1      # more than 8 tokens
     assert m.moe_launch_count(cfg, 4, 7, m.MOE_PATH_AUTO) == -1          # no such mode
     assert m.moe_launch_count(cfg, 0, SC, m.MOE_PATH_AUTO) == -1
+
+
+def test_gdn_scan_validation_before_launch():
+    """The scan refuses counts below 1, null or misaligned pointers and head
+    sizes other than 128 before launching anything."""
+    import bit_dequant_expert_b200 as m
+
+    def call(B=1, T=4, Hk=2, Hv=4, dk=128, dv=128, q=FAKE, g=FAKE, s_out=FAKE, o=FAKE):
+        return m.gdn_scan(B, T, Hk, Hv, dk, dv, q, FAKE, FAKE, g, FAKE, 0.1, FAKE, s_out, o, stream=0,
+                          raise_on_error=False)
+
+    assert call(B=0) == m.MOE_ERR_INVALID_ARG
+    assert call(T=0) == m.MOE_ERR_INVALID_ARG
+    assert call(q=None) == m.MOE_ERR_INVALID_ARG
+    assert call(q=FAKE + 8) == m.MOE_ERR_INVALID_ARG
+    assert call(o=FAKE + 2) == m.MOE_ERR_INVALID_ARG
+    assert call(g=FAKE + 2) == m.MOE_ERR_INVALID_ARG
+    assert call(s_out=None) == m.MOE_ERR_INVALID_ARG
+    assert call(dk=64) == m.MOE_ERR_UNSUPPORTED
+    assert call(dv=256) == m.MOE_ERR_UNSUPPORTED
+    assert call(Hk=3, Hv=4) == m.MOE_ERR_UNSUPPORTED
