@@ -56,12 +56,15 @@ constexpr int kDnSlots = 2;                     // down ring: one unit's down co
 constexpr int kMaxSlots = 1 + 8 * kMaxT;        // active experts: shared + 8 per token
 constexpr int kSmemLimit = 232448;              // dynamic shared memory per block (227 KB)
 constexpr int kRouterRows = 2;                  // router rows per CTA (experts b and b + grid size)
+constexpr int kExtraBars = 7;                   // mbarriers besides the two rings
 
 struct DecLayout {
     int gu_box;     // gate/up codes box: 16 rows x H/2 bytes
     int gu_sbb;     // gate/up (scale, bias) box slot: 16 rows x H/16 bytes, 1 KB aligned
     int gu_slots;   // gate/up ring depth
     int dn_box;     // one unit's down codes: H rows x 16 bytes
+    int sb_tma;     // 1: the down (scale, bias) words arrive as one TMA box of H rows x 16 bytes (I >= 256)
+    int dsb_bytes;  // their landing area: H x 16 bytes by TMA, else H words by cp.async
     int xs;         // x row stride (bytes)
     int off_gu, off_gusb, off_dn, off_dsb, off_x, off_sx, off_red, off_hs, off_rt, off_tab, off_bar, total;
 };
@@ -85,29 +88,30 @@ struct DecTab {
 __host__ __device__ inline int round_up(int v, int a) { return (v + a - 1) / a * a; }
 
 DecLayout dec_layout(int H, int I, int T) {
-    (void)I;
     DecLayout L;
     L.gu_box = 8 * H;
     L.gu_sbb = round_up(H, 1024);
     L.dn_box = 16 * H;
+    L.sb_tma = I >= 256 ? 1 : 0;
+    L.dsb_bytes = L.sb_tma ? 16 * H : 4 * H;
     L.xs = 2 * H + 16;
-    const int fixed = kDnSlots * L.dn_box + 4 * H + round_up(T * L.xs, 128) + (H / 64) * kMaxT * 4 +
+    const int fixed = kDnSlots * L.dn_box + L.dsb_bytes + round_up(T * L.xs, 128) + (H / 64) * kMaxT * 4 +
                       kWarps * 32 * 16 + 2 * kMaxT * 32 * 2 + kRouterRows * 2 * H + round_up((int)sizeof(DecTab), 128) +
-                      (2 * kMaxGuSlots + 2 * kDnSlots + 5) * 8 + 6 * 128;
+                      (2 * kMaxGuSlots + 2 * kDnSlots + kExtraBars) * 8 + 6 * 128;
     L.gu_slots = (kSmemLimit - 1024 - fixed) / (L.gu_box + L.gu_sbb);
     if (L.gu_slots > kMaxGuSlots) L.gu_slots = kMaxGuSlots;
     L.off_gu = 0;
     L.off_gusb = L.off_gu + L.gu_slots * L.gu_box;
     L.off_dn = L.off_gusb + L.gu_slots * L.gu_sbb;
     L.off_dsb = L.off_dn + kDnSlots * L.dn_box;
-    L.off_x = round_up(L.off_dsb + 4 * H, 128);
+    L.off_x = round_up(L.off_dsb + L.dsb_bytes, 128);
     L.off_sx = round_up(L.off_x + T * L.xs, 128);
     L.off_red = round_up(L.off_sx + (H / 64) * kMaxT * 4, 128);
     L.off_hs = round_up(L.off_red + kWarps * 32 * 16, 128);
     L.off_rt = round_up(L.off_hs + 2 * kMaxT * kJ * 2, 128);
     L.off_tab = round_up(L.off_rt + kRouterRows * 2 * H, 128);
     L.off_bar = round_up(L.off_tab + (int)sizeof(DecTab), 8);
-    L.total = L.off_bar + (2 * kMaxGuSlots + 2 * kDnSlots + 5) * 8;
+    L.total = L.off_bar + (2 * kMaxGuSlots + 2 * kDnSlots + kExtraBars) * 8;
     return L;
 }
 
@@ -165,7 +169,8 @@ __device__ __forceinline__ unsigned long long tag_word(uint32_t epoch, float v) 
 template <int kH, bool kRoute>
 __global__ void __launch_bounds__(kThreads, 1)
     k_decode(const __grid_constant__ CUtensorMap gu_map, const __grid_constant__ CUtensorMap gsb_map,
-             const __grid_constant__ CUtensorMap dn_map, const DecArgs da) {
+             const __grid_constant__ CUtensorMap dn_map, const __grid_constant__ CUtensorMap dsb_map,
+             const DecArgs da) {
     constexpr int kNG = kH / 64;                 // (scale, bias) groups per gate/up row
     constexpr int kNGW = kNG / 4;                // groups per K-quarter warp
     constexpr int kNCH = kH / 256;               // 128-byte lines per gate/up code row
@@ -200,6 +205,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* list_ready = rt_full + 2;   // the active list is in shared memory (producer lane 0 waits)
     uint64_t* zt_ready = rt_full + 3;     // the launch number is in shared memory (the logits' tag)
     uint64_t* zeroed = rt_full + 4;       // this CTA's slice of y_acc is cleared (producer lane 0 waits)
+    uint64_t* dsb_full = rt_full + 5;     // the unit's down (scale, bias) box landed (TMA form)
+    uint64_t* dsb_empty = rt_full + 6;    // and was read by every compute warp
     uint8_t* xs = smem + L.off_x;                                    // [T][kH] bf16, split order
     float* sx = reinterpret_cast<float*>(smem + L.off_sx);           // [kNG][kMaxT] group sums of x
     float4* red = reinterpret_cast<float4*>(smem + L.off_red);       // [kWarps][32]
@@ -220,18 +227,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(list_ready, 1);
         mbar_init(zt_ready, 1);
         mbar_init(zeroed, 1);
+        mbar_init(dsb_full, 1);
+        mbar_init(dsb_empty, kWarps);
         fence_mbar_init();
     }
     if (warp == kWarps && lane == 0) {
         prefetch_tensormap(&gu_map);
         prefetch_tensormap(&gsb_map);
         prefetch_tensormap(&dn_map);
+        if (L.sb_tma) prefetch_tensormap(&dsb_map);
     }
     __syncthreads();
 
     // ---- loads (producer lane 0)
     // gate/up boxes of a unit (expert e, column block jb), then its down columns
-    int gu_n = 0, gu_cs = 0, gu_ph = 0, dn_n = 0;
+    int gu_n = 0, gu_cs = 0, gu_ph = 0, dn_n = 0, sb_n = 0;
+    // Producer lane 0: the first reductions into y_acc wait until every CTA has
+    // cleared its slice.  release_zero polls the launch counter for that and
+    // opens zero_done; it must run before any load waits on a down phase.
+    bool released = false;
+    auto release_zero = [&]() {
+        const unsigned long long target = tab.zero_target;
+        const uint64_t t0 = globaltimer_ns();
+        while (ld_relaxed_u64(da.launches) < target) {
+            if (globaltimer_ns() - t0 > 200000000ull) {
+                set_error(a.err, MOE_ERR_TIMEOUT);
+                break;
+            }
+            __nanosleep(64);
+        }
+        __threadfence();
+        mbar_arrive(zero_done);
+        released = true;
+    };
     auto issue_unit = [&](int e, int jb) {
         for (int p = 0; p < 4; ++p) {
             if (gu_n >= gus) mbar_wait_bounded(&gu_empty[gu_cs], (gu_ph - 1) & 1, a.err);
@@ -249,16 +277,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&dn_full[ds], L.dn_box);
         tma_load_4d(smem + L.off_dn + ds * L.dn_box, &dn_map, 0, 0, e * (kH / 256), jb, &dn_full[ds]);
         ++dn_n;
+        if (L.sb_tma) {
+            // every row's 16-byte piece holding word jb / 2 of its (scale, bias) row; one slot
+            if (sb_n >= 1) {
+                if (!released) release_zero();   // the previous unit's down phase may wait on it
+                mbar_wait_bounded(dsb_empty, (sb_n - 1) & 1, a.err);
+            }
+            mbar_arrive_expect_tx(dsb_full, (uint32_t)L.dsb_bytes);
+            tma_load_4d(smem + L.off_dsb, &dsb_map, 0, 0, e * (kH / 256), (jb >> 1) >> 2, dsb_full);
+            ++sb_n;
+        }
     };
-    // weights do not depend on earlier grids: the shared expert's unit and the router rows go first
+    // weights do not depend on earlier grids: the router rows and the shared expert's unit go first
     const int nr = kRoute ? min((E - b + G - 1) / G, kRouterRows) : 0;
     if (warp == kWarps && lane == 0) {
-        if (early_unit) issue_unit(E, b);
+        // the router rows first: every CTA's logits wait on them, and the slowest CTA's decide the top-k
         if (kRoute) {
             mbar_arrive_expect_tx(rt_full, (uint32_t)(nr * 2 * kH));
             for (int r = 0; r < nr; ++r)
                 bulk_load(smem + L.off_rt + r * 2 * kH, da.r.w_router + (size_t)(b + r * G) * kH, 2 * kH, rt_full);
         }
+        if (early_unit) issue_unit(E, b);
     }
     const int r_e = b + warp * G;
     const bool r_on = kRoute && warp < nr;
@@ -288,12 +327,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool zero_seen = false;
     auto compute_unit = [&](int k, int s, int jb) {
         const int e = tab.slot_e[s];
-        // the down (scale, bias) word of every row for this block's group of I
-        {
+        // the down (scale, bias) word of every row for this block's group of I (the
+        // TMA form lands with the unit's other boxes)
+        if (!L.sb_tma) {
             const uint32_t* src = reinterpret_cast<const uint32_t*>(a.d_sb) + (size_t)e * kH * (I >> 6) + (jb >> 1);
             for (int n = tid; n < kH; n += kWarps * 32) cp_async4(smem_u32(dsb + n), src + (size_t)n * (I >> 6));
-            cp_async_commit();
         }
+        cp_async_commit();
         // ---- gate/up
         while (cu_n < 4 * k + p_box) {
             ++cu_n;
@@ -371,6 +411,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float hs1 = (tab.hsum[k & 1][0][t1c] + tab.hsum[k & 1][1][t1c]) +
                           (tab.hsum[k & 1][2][t1c] + tab.hsum[k & 1][3][t1c]);
         const float w0 = tab.wsel[s][2 * c], w1 = tab.wsel[s][2 * c + 1];
+        if (L.sb_tma) mbar_wait_bounded(dsb_full, k & 1, a.err);
+        // row n's word: a 16-byte piece per row holding word (jb / 2) % 4 (TMA form), else one word per row
+        const uint8_t* sbrow = reinterpret_cast<const uint8_t*>(dsb) + (L.sb_tma ? 4 * ((jb >> 1) & 3) : 0);
+        const int sbs = L.sb_tma ? 16 : 4;
         if (!zero_seen) {   // the first reduction into y_acc waits until every CTA cleared its slice
             mbar_wait_bounded(zero_done, 0, a.err);
             zero_seen = true;
@@ -385,8 +429,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_bf16_16816(d, nib(ca, 0), nib(cb, 0), nib(ca, 1), nib(cb, 1), hv.x, hv.y);
             mma_bf16_16816(d, nib(ca, 2), nib(cb, 2), nib(ca, 3), nib(cb, 3), hv.z, hv.w);
             float sa, ba, sb2, bb2;
-            sb_factor(dsb[n], sa, ba);
-            sb_factor(dsb[n + 8], sb2, bb2);
+            sb_factor(lds32(sbrow + n * sbs), sa, ba);
+            sb_factor(lds32(sbrow + (n + 8) * sbs), sb2, bb2);
             // w (s D + (b - 128 s) sum(h)) for rows n (d0, d1) and n + 8 (d2, d3), tokens 2c, 2c+1
             const float v0 = w0 != 0.0f ? w0 * fmaf(sa, d[0], ba * hs0) : 0.0f;
             const float v2 = w0 != 0.0f ? w0 * fmaf(sb2, d[2], bb2 * hs0) : 0.0f;
@@ -425,7 +469,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&dn_empty[ds]);
+        if (lane == 0) {
+            mbar_arrive(&dn_empty[ds]);
+            if (L.sb_tma) mbar_arrive(dsb_empty);
+        }
         named_barrier(1, kWarps * 32);   // hs, dsb and the sums free for the next unit
     };
 
@@ -672,37 +719,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait_bounded(zeroed, 0, a.err);
             __threadfence();
             red_add_relaxed_u64(da.launches, 1ull);
-            // every CTA counted: release the first reductions into y_acc
-            auto release_zero = [&]() {
-                const unsigned long long target = tab.zero_target;
-                const uint64_t t0 = globaltimer_ns();
-                while (ld_relaxed_u64(da.launches) < target) {
-                    if (globaltimer_ns() - t0 > 200000000ull) {
-                        set_error(a.err, MOE_ERR_TIMEOUT);
-                        break;
-                    }
-                    __nanosleep(64);
-                }
-                __threadfence();
-                mbar_arrive(zero_done);
-            };
             // the fused layer's shared-expert unit reduces into y_acc before the active
             // list exists; otherwise units 0 and 1 go first (their loads never wait on a
             // reduction), then the release, then the rest
-            bool released = false;
-            if (kRoute && early_unit) {
-                release_zero();
-                released = true;
-            }
+            if (kRoute && early_unit) release_zero();
             mbar_wait_bounded(list_ready, 0, a.err);
             const int A = tab.A;
             int u = b, s = b >> (lgI - 5), jb = b & (NJ - 1), k = 0;
             const int dsl = G >> (lgI - 5), dj = G & (NJ - 1);
             for (; u < A * NJ; u += G, ++k) {
-                if (!released && k == 2) {
-                    release_zero();
-                    released = true;
-                }
+                if (!released && k == 2) release_zero();
                 if (!(u == b && early_unit)) issue_unit(tab.slot_e[s], jb);
                 s += dsl;
                 jb += dj;
@@ -796,9 +822,25 @@ bool make_dn_map(CUtensorMap* m, const FfnArgs& a) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Down (scale, bias) words as a 4-D view (4 words = one 16-byte piece of a
+// row's I/64 words, row of a 256-row band, band of all experts' rows, piece);
+// one box = the H rows of one expert, the piece holding a unit's word.
+bool make_dsb_map(CUtensorMap* m, const FfnArgs& a) {
+    EncodeTiled enc = dec_encode_fn();
+    if (!enc) return false;
+    const uint64_t row = (uint64_t)a.I / 16;   // bytes of one row's words
+    const cuuint64_t dims[4] = {4, 256, (cuuint64_t)(a.E + 1) * (a.H / 256), (cuuint64_t)(a.I / 256)};
+    const cuuint64_t strides[3] = {row, 256 * row, 16};
+    const cuuint32_t box[4] = {4, 256, (cuuint32_t)(a.H / 256), 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, const_cast<uint16_t*>(a.d_sb), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int kH, bool kRoute>
 cudaError_t launch_dec_h(const DecArgs& da, const CUtensorMap& gu_map, const CUtensorMap& gsb_map,
-                         const CUtensorMap& dn_map, cudaStream_t st) {
+                         const CUtensorMap& dn_map, const CUtensorMap& dsb_map, cudaStream_t st) {
     static int done[64] = {0};
     const int smem = da.L.total + 1024;
     cudaError_t ce = set_smem_once(k_decode<kH, kRoute>, smem, done);
@@ -822,18 +864,23 @@ cudaError_t launch_dec_h(const DecArgs& da, const CUtensorMap& gu_map, const CUt
     attr[1].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, k_decode<kH, kRoute>, gu_map, gsb_map, dn_map, da);
+    return cudaLaunchKernelEx(&cfg, k_decode<kH, kRoute>, gu_map, gsb_map, dn_map, dsb_map, da);
 }
 
 template <bool kRoute>
 cudaError_t launch_dec(const DecArgs& da, cudaStream_t st) {
-    CUtensorMap gu_map, gsb_map, dn_map;
+    CUtensorMap gu_map, gsb_map, dn_map, dsb_map;
     if (!make_gu_map(&gu_map, da.f) || !make_gsb_map(&gsb_map, da.f) || !make_dn_map(&dn_map, da.f))
         return cudaErrorInvalidValue;
+    if (da.L.sb_tma) {
+        if (!make_dsb_map(&dsb_map, da.f)) return cudaErrorInvalidValue;
+    } else {
+        dsb_map = dn_map;   // not read
+    }
     switch (da.f.H) {
-        case 512: return launch_dec_h<512, kRoute>(da, gu_map, gsb_map, dn_map, st);
-        case 1024: return launch_dec_h<1024, kRoute>(da, gu_map, gsb_map, dn_map, st);
-        case 2048: return launch_dec_h<2048, kRoute>(da, gu_map, gsb_map, dn_map, st);
+        case 512: return launch_dec_h<512, kRoute>(da, gu_map, gsb_map, dn_map, dsb_map, st);
+        case 1024: return launch_dec_h<1024, kRoute>(da, gu_map, gsb_map, dn_map, dsb_map, st);
+        case 2048: return launch_dec_h<2048, kRoute>(da, gu_map, gsb_map, dn_map, dsb_map, st);
         default: return cudaErrorInvalidValue;
     }
 }
