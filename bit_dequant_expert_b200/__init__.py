@@ -44,6 +44,7 @@ EXPORTED = (
     "moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permute", "moe_expert_ffn",
     "moe_expert_ffn_path", "moe_combine", "moe_get_device_error", "moe_status_string", "moe_launch_count",
     "moe_permute_static", "moe_decode_layer", "moe_wait_selftest", "moe_gather_rows", "gdn_scan",
+    "moe_router_logits",
 )
 
 MOE_STATIC_MAX_TOKENS = 16384
@@ -68,6 +69,8 @@ _lib.moe_workspace_init.restype = _I32
 _lib.moe_workspace_init.argtypes = [_P, ctypes.c_size_t, _P]
 _lib.moe_route.restype = _I32
 _lib.moe_route.argtypes = [_CFG, _I32, _P, _P, _P, _P, ctypes.c_int64, _P, _P, _P, _P, ctypes.c_size_t, _P]
+_lib.moe_router_logits.restype = _I32
+_lib.moe_router_logits.argtypes = [_CFG, _I32, _P, _P, _P, ctypes.c_int64, _P, _P, ctypes.c_size_t, _P]
 _lib.moe_permute.restype = _I32
 _lib.moe_permute.argtypes = [_CFG, _I32, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.moe_expert_ffn.restype = _I32
@@ -149,6 +152,14 @@ def moe_route(cfg, T, x, w_router, logits_in, logit_bias, logit_bias_row_stride,
                         logit_bias_row_stride, _ptr(topk_idx), _ptr(topk_w), _ptr(counts), _ptr(ws), n,
                         _stream(stream))
     return _check(st, "moe_route", raise_on_error)
+
+
+def moe_router_logits(cfg, T, x, w_router, logit_bias, logit_bias_row_stride, logits, ws, ws_bytes=None,
+                      stream=None, raise_on_error=True) -> int:
+    n = _nbytes(ws) if ws_bytes is None else ws_bytes
+    st = _lib.moe_router_logits(ctypes.byref(cfg), T, _ptr(x), _ptr(w_router), _ptr(logit_bias),
+                                logit_bias_row_stride, _ptr(logits), _ptr(ws), n, _stream(stream))
+    return _check(st, "moe_router_logits", raise_on_error)
 
 
 def moe_permute(cfg, T, topk_idx, counts, offsets, row_to_pair, pair_to_row, ws, ws_bytes=None, stream=None,

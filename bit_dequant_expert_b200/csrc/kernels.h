@@ -94,6 +94,8 @@ struct GdnArgs {
 bool gdn_scan_supported(const GdnArgs& a);
 cudaError_t launch_gdn_scan(const GdnArgs& a, cudaStream_t st);
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t st);
+// The logits alone (+ bias) into a.logits_ws; zeroes a.counts when non-null.
+cudaError_t launch_router_logits(const RouterArgs& a, cudaStream_t st);
 size_t permute_ws_bytes(int T, int E, int K);
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st);
 cudaError_t launch_ffn_simt(const FfnArgs& a, cudaStream_t st);

@@ -134,6 +134,30 @@ int32_t moe_route(const moe_config_t* cfg, int32_t T, const uint16_t* x, const u
     return cuda_status(launch_router(a, (cudaStream_t)stream));
 }
 
+int32_t moe_router_logits(const moe_config_t* cfg, int32_t T, const uint16_t* x, const uint16_t* w_router,
+                          const float* logit_bias, int64_t logit_bias_row_stride, float* logits, void* ws,
+                          size_t ws_bytes, void* stream) {
+    if (!ws) return MOE_ERR_WORKSPACE;
+    int32_t st = check_common(cfg, T, ws, ws_bytes);
+    if (st) return st;
+    if (!routing_shape_ok(cfg)) return MOE_ERR_UNSUPPORTED;
+    if (!x || !w_router || !logits) return MOE_ERR_INVALID_ARG;
+    if (logit_bias_row_stride < 0) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(logit_bias, 4) || !aligned(logits, 8))
+        return MOE_ERR_INVALID_ARG;
+    RouterArgs a = {};
+    a.T = T;
+    a.H = cfg->hidden;
+    a.E = cfg->num_experts;
+    a.x = x;
+    a.w_router = w_router;
+    a.bias = logit_bias;
+    a.bias_stride = logit_bias_row_stride;
+    a.logits_ws = logits;
+    a.err = err_word(ws);
+    return cuda_status(launch_router_logits(a, (cudaStream_t)stream));
+}
+
 int32_t moe_permute(const moe_config_t* cfg, int32_t T, const int32_t* topk_idx, const int32_t* counts,
                     int32_t* offsets, int32_t* row_to_pair, int32_t* pair_to_row, void* ws, size_t ws_bytes,
                     void* stream) {

@@ -103,11 +103,16 @@ def key(seed: int, tensor: int, layer: int) -> int:
     return int(lib().gen_key(seed, tensor, layer))
 
 
+def make_router(spec: LayerSpec, layer: int = 0) -> np.ndarray:
+    """Router weights bf16 [E, H] of one layer (the same as make_weights')."""
+    return normal_bf16(key(spec.seed, TID_ROUTER, layer), 0.02, spec.E * spec.H).reshape(spec.E, spec.H)
+
+
 def make_weights(spec: LayerSpec, layer: int = 0) -> dict:
     """Router and expert weights of one layer (E routed experts + 1 shared)."""
     E, H, I, G = spec.E, spec.H, spec.I, spec.G
     s = spec.seed
-    w_router = normal_bf16(key(s, TID_ROUTER, layer), 0.02, E * H).reshape(E, H)
+    w_router = make_router(spec, layer)
     gu_codes = np.empty((E + 1, 2 * I, H // 8), dtype=np.uint32)
     lib().gen_codes(key(s, TID_GU_CODES, layer), _ptr(gu_codes), gu_codes.size)
     gu_sb = np.empty((E + 1, 2 * I, H // G, 2), dtype=np.uint16)

@@ -133,6 +133,19 @@ int32_t moe_route(const moe_config_t* cfg, int32_t T, const uint16_t* x, const u
                   void* stream);
 
 /*
+ * The router logits alone: logits fp32 [T, E] (device, caller-owned, 8-byte
+ * aligned) = x . w_router^T in the contract order above, + logit_bias when
+ * given; the same values moe_route selects from.  x, w_router, logit_bias and
+ * the stride as for moe_route; the workspace carries the error word (a
+ * bounded wait that expires sets MOE_ERR_TIMEOUT there).  Returns
+ * MOE_ERR_INVALID_ARG for a null or misaligned pointer or a negative stride,
+ * else as moe_route.
+ */
+int32_t moe_router_logits(const moe_config_t* cfg, int32_t T, const uint16_t* x, const uint16_t* w_router,
+                          const float* logit_bias, int64_t logit_bias_row_stride, float* logits, void* ws,
+                          size_t ws_bytes, void* stream);
+
+/*
  * Token permutation: stable expert-major order of the T*k (token, slot)
  * pairs, pair p = t*k + slot.
  *   counts      nullable int32 [E] from moe_route; when given it is checked

@@ -20,7 +20,7 @@ def declared_functions():
 def test_header_declares_the_layer_calls():
     names = declared_functions()
     for n in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_workspace_size",
-              "moe_get_device_error", "moe_gather_rows", "gdn_scan"):
+              "moe_get_device_error", "moe_gather_rows", "gdn_scan", "moe_router_logits"):
         assert n in names
 
 
@@ -83,6 +83,18 @@ def test_host_validation_before_launch():
     assert st == m.MOE_ERR_INVALID_ARG      # pairs mode with a shared expert needs out1
     st = m.moe_combine(cfg, 64, 1, FAKE, FAKE, None, FAKE, FAKE, stream=0, raise_on_error=False)
     assert st == m.MOE_ERR_INVALID_ARG
+    def logits(T=64, x=FAKE, out=FAKE, bias=None, stride=0, ws=FAKE, c=cfg):
+        return m.moe_router_logits(c, T, x, FAKE, bias, stride, out, ws, ws_bytes=need, stream=0,
+                                   raise_on_error=False)
+
+    assert logits(T=0) == m.MOE_ERR_INVALID_ARG
+    assert logits(x=None) == m.MOE_ERR_INVALID_ARG
+    assert logits(x=FAKE + 8) == m.MOE_ERR_INVALID_ARG
+    assert logits(out=FAKE + 4) == m.MOE_ERR_INVALID_ARG
+    assert logits(bias=FAKE + 2) == m.MOE_ERR_INVALID_ARG
+    assert logits(bias=FAKE, stride=-1) == m.MOE_ERR_INVALID_ARG
+    assert logits(ws=None) == m.MOE_ERR_WORKSPACE
+    assert logits(c=m.config(num_experts=128, top_k=1, has_shared=0)) == m.MOE_ERR_UNSUPPORTED
     assert m.moe_get_device_error(None, 0) == m.MOE_ERR_WORKSPACE
     assert m.moe_status_string(m.MOE_ERR_NONFINITE) == "MOE_ERR_NONFINITE"
 
