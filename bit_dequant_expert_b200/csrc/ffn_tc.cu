@@ -9,9 +9,13 @@
 // expanded array never touches memory: +77.4% prefill at 512 tokens).
 //
 // One persistent kernel, launched once for gate/up (+SwiGLU) and once for
-// down (+weighted combine).  A tile is 128 weight rows (MMA M) x up to 128
+// down (+weighted combine).  A tile is 128 weight rows (MMA M) x up to nt
 // token rows (MMA N) of one expert; K runs in 128-input stages (two (scale,
-// bias) groups), three stages in flight.  Roles:
+// bias) groups), three stages in flight.  nt is 128, or 80 when the experts
+// hold few rows each (T k <= 96 E): one thread's stream of tcgen05.mma
+// instructions runs at about one per 66 ns for any N up to 256, so narrow
+// tiles are bound by the issue rate, and then the two 64-input halves of
+// every stage go to two issuing threads with an accumulator each.  Roles:
 //   warp 0       TMA of the codes (128 rows x 256 inputs per 16 KB box, two
 //                stages, 128B-swizzled) and of each tile's (scale, bias) rows;
 //   warps 2-3    one 3-D TMA box per stage of the B operand: the tile's token
@@ -22,10 +26,14 @@
 //   warps 4-11   dequantise codes to bf16 (scale * q + bias; a code word
 //                gives the nibble pairs (j, j+4), and x and h are stored in
 //                that order inside every 8 inputs) and write them as the A
-//                operand straight into tensor memory (tcgen05.st);
-//   warp 1       one thread issues 8 tcgen05.mma (K = 16 each) per stage into
-//                one of two TMEM accumulators and commits to mbarriers;
-//   warps 12-15  epilogue from TMEM: SwiGLU (gate and up rows interleaved on
+//                operand straight into tensor memory (tcgen05.st); warps
+//                4-7 the first 64 inputs of a stage, 8-11 the other 64;
+//   warps 1, 16  one thread each issues the tcgen05.mma (K = 16 each) of a
+//                stage (warp 1 all 8 when nt = 128; 4 each, one 64-input
+//                half, when nt = 80) into the tile's accumulator(s), double-
+//                buffered, and commits to mbarriers;
+//   warps 12-15  epilogue from TMEM (the sum of the two K-half accumulators
+//                when split): SwiGLU (gate and up rows interleaved on
 //                adjacent TMEM lanes) -> h in bf16, or bf16 rows (paired
 //                32-bit stores) / w * y added into y_acc (fp32 red).
 // Every wait is bounded (error word MOE_ERR_TIMEOUT, never a hang).
@@ -39,15 +47,23 @@ namespace moe {
 
 namespace {
 
-constexpr int kThreads = 512;
-constexpr int kNT = 128;                 // token rows per tile (MMA N, max)
-static_assert(kNT % 64 == 0, "the column-table builders cover kNT columns with 64 threads");
+constexpr int kThreads = 544;
+// Token rows per tile (MMA N, max), chosen per launch: 128 with one MMA
+// issuer and two accumulator buffers, or 80 with the K halves of every chunk
+// on two issuers (four accumulators: two K halves, double-buffered); either
+// way the accumulators end below column kACol0 and the A stages fill the
+// rest of the 512 TMEM columns.
+constexpr int kNTWide = 128;
+constexpr int kNTSplit = 80;
+static_assert(kNTSplit % 16 == 0, "MMA N is a multiple of 16");
 constexpr int kBK = 128;                 // inputs per chunk = two (scale, bias) groups
 constexpr int kStages = 3;              // B ring and TMEM A stages (128 inputs each)
 constexpr int kCStages = 4;             // codes ring
 constexpr int kCodesStage = 128 * 128;  // 128 rows x 256 nibbles (four chunks), 128B-swizzled
-constexpr int kBStage = kNT * 2 * 128;   // two 64-input halves of kNT rows x 64 bf16
-constexpr int kACol0 = 2 * kNT;          // TMEM: two fp32 accumulators, then the A stages
+constexpr int kBRows = 128;              // rows of the larger B box (tiles of more than 64 rows)
+constexpr int kBStage = kBRows * 2 * 128;   // two 64-input halves of up to 128 rows x 64 bf16
+constexpr int kACol0 = 4 * kNTSplit;     // TMEM: the accumulators, then the A stages
+static_assert(2 * kNTWide <= kACol0, "TMEM budget");
 constexpr int kAStageCols = kBK / 2;     // bf16 pairs per 32-bit column
 constexpr int kTmemCols = 512;
 constexpr int kTabs = 4;                 // column tables in flight (down epilogue)
@@ -58,10 +74,10 @@ struct Smem {
     uint8_t b[kStages][kBStage];                 // offset 0, 1024-aligned
     uint8_t codes[kCStages][kCodesStage];
     uint32_t sbs[2][kSbBytes / 4];               // per-tile (scale, bias) rows, double-buffered
-    uint64_t full[kStages], a_full[kStages], mma_done[kStages], cfull[kCStages], cempty[kCStages];
+    uint64_t full[kStages], a_full[2][kStages], mma_done[kStages], cfull[kCStages], cempty[kCStages];
     uint64_t acc_full[2], acc_empty[2], tab_full[kTabs], tab_empty[kTabs], sb_full[2], sb_empty[2];
-    int tok[kTabs][kNT];
-    float w[kTabs][kNT];
+    int tok[kTabs][kNTWide];
+    float w[kTabs][kNTWide];
     int pre[260];
     int off[260];                                // offsets[0..E], cached
     uint32_t tmem_base;
@@ -70,6 +86,8 @@ struct Smem {
 struct TcArgs {
     FfnArgs f;
     int gateup;      // 1: gate/up + SwiGLU; 0: down + combine
+    int nt;          // token rows per tile: kNTSplit (ksplit) or kNTWide
+    int ksplit;      // 1: the K halves of every chunk on two MMA issuers
 };
 
 struct Tile {
@@ -83,7 +101,7 @@ __device__ __forceinline__ int tiles_per_block_row(const FfnArgs& a, int gateup)
 
 // Prefix of tiles per expert: pre[e] first tile of expert e, pre[E] first
 // shared tile, pre[E+1] total.  blockDim.x >= E.
-__device__ void tile_prefix(const FfnArgs& a, int gateup, int* pre, int* off) {
+__device__ void tile_prefix(const FfnArgs& a, int gateup, int nt, int* pre, int* off) {
     __shared__ int warp_tot[32];
     const int MB = tiles_per_block_row(a, gateup);
     const int e = threadIdx.x;
@@ -94,7 +112,7 @@ __device__ void tile_prefix(const FfnArgs& a, int gateup, int* pre, int* off) {
             set_error(a.err, MOE_ERR_BOUNDS);
             lo = hi = 0;
         }
-        tiles = (hi - lo + kNT - 1) / kNT * MB;
+        tiles = (hi - lo + nt - 1) / nt * MB;
         off[e] = lo;
         if (e == a.E - 1) off[a.E] = hi;
     }
@@ -113,12 +131,13 @@ __device__ void tile_prefix(const FfnArgs& a, int gateup, int* pre, int* off) {
     if (threadIdx.x == blockDim.x - 1) {
         const int routed = base + inc;
         pre[a.E] = routed;
-        pre[a.E + 1] = routed + (a.has_shared ? (a.T + kNT - 1) / kNT * MB : 0);
+        pre[a.E + 1] = routed + (a.has_shared ? (a.T + nt - 1) / nt * MB : 0);
     }
     __syncthreads();
 }
 
-__device__ __forceinline__ Tile decode_tile(const FfnArgs& a, int gateup, const int* pre, const int* off, int t) {
+__device__ __forceinline__ Tile decode_tile(const FfnArgs& a, int gateup, int nt, const int* pre, const int* off,
+                                            int t) {
     const int MB = tiles_per_block_row(a, gateup);
     Tile tl;
     int e;
@@ -137,12 +156,12 @@ __device__ __forceinline__ Tile decode_tile(const FfnArgs& a, int gateup, const 
     tl.e = e;
     tl.mb = local % MB;
     if (e == a.E) {
-        tl.r0 = tb * kNT;
-        tl.nr = min(kNT, a.T - tl.r0);
+        tl.r0 = tb * nt;
+        tl.nr = min(nt, a.T - tl.r0);
         tl.hrow0 = (size_t)a.T * a.K + tl.r0;
     } else {
-        tl.r0 = off[e] + tb * kNT;
-        tl.nr = min(kNT, (e + 1 < a.E ? off[e + 1] : off[a.E]) - tl.r0);
+        tl.r0 = off[e] + tb * nt;
+        tl.nr = min(nt, (e + 1 < a.E ? off[e + 1] : off[a.E]) - tl.r0);
         tl.hrow0 = tl.r0;
     }
     tl.npad = (tl.nr + 15) & ~15;
@@ -164,6 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const FfnArgs& a = ta.f;
     const int gateup = ta.gateup;
+    const int nt = ta.nt, ksplit = ta.ksplit;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int K = gateup ? a.H : a.I;            // reduction length of this GEMM
     const int KC = K / kBK;                      // chunks per tile
@@ -180,15 +200,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.full[s], 1);
-            mbar_init(&sm.a_full[s], 8);
-            mbar_init(&sm.mma_done[s], 1);
+            mbar_init(&sm.a_full[0][s], 4);
+            mbar_init(&sm.a_full[1][s], 4);
+            mbar_init(&sm.mma_done[s], ksplit ? 2 : 1);
         }
         for (int s = 0; s < kCStages; ++s) {
             mbar_init(&sm.cfull[s], 1);
             mbar_init(&sm.cempty[s], 8);
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&sm.acc_full[b], 1);
+            mbar_init(&sm.acc_full[b], ksplit ? 2 : 1);
             mbar_init(&sm.acc_empty[b], 4);
         }
         for (int b = 0; b < kTabs; ++b) {
@@ -214,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (size_t q = lo + tid; q < hi; q += kThreads)
             reinterpret_cast<float4*>(a.y_acc)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    tile_prefix(a, gateup, sm.pre, sm.off);   // contains __syncthreads
+    tile_prefix(a, gateup, nt, sm.pre, sm.off);   // contains __syncthreads
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     const int ntiles = sm.pre[a.E + 1];
@@ -225,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // a stage is refilled once its chunks were dequantised.
         uint32_t it = 0, lt = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
-            const Tile tl = decode_tile(a, gateup, sm.pre, sm.off, t);
+            const Tile tl = decode_tile(a, gateup, nt, sm.pre, sm.off, t);
             if (sb_tma && lane == 0) {
                 const int buf = lt & 1;
                 if (lt >= 2) mbar_wait_bounded(&sm.sb_empty[buf], ((lt >> 1) - 1) & 1, a.err);
@@ -255,20 +276,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
             }
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+    } else if (warp == 1 || warp == 16) {
+        // ------------------------------------------------------------ MMA issuers
+        // One thread of warp 1 issues the MMAs of the first 64 inputs of every
+        // chunk into K-half accumulator 0 of the tile's buffer, one of warp 16
+        // those of the other 64 into accumulator 1: a thread's tcgen05.mma
+        // stream runs at about one instruction per 66 ns whatever N is, so two
+        // streams raise the rate for the narrow token tiles; the epilogue adds
+        // the two accumulators.
+        const int h = warp == 1 ? 0 : 1;
+        // one issuer (warp 1) for the whole chunk when the K halves are not split
+        const int j0 = ksplit ? 4 * h : 0, j1 = ksplit ? 4 * h + 4 : 8;
+        if (lane == 0 && (ksplit || h == 0)) {
             uint32_t lt = 0, par = 0;
             int s = 0;   // ring stage and its phase, advanced per chunk
             for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
-                const Tile tl = decode_tile(a, gateup, sm.pre, sm.off, t);
+                const Tile tl = decode_tile(a, gateup, nt, sm.pre, sm.off, t);
                 const int ab = lt & 1;
                 if (lt >= 2) mbar_wait_bounded(&sm.acc_empty[ab], ((lt >> 1) - 1) & 1, a.err);
                 tc_fence_after();
                 const uint32_t idesc = idesc_bf16_f32(128, tl.npad);
-                const uint32_t d_tmem = tmem + ab * kNT;
+                const uint32_t d_tmem = tmem + (ksplit ? (2 * ab + h) * nt : ab * nt);
                 for (int kc = 0; kc < KC; ++kc) {
-                    mbar_wait_bounded(&sm.a_full[s], par, a.err);
+                    if (ksplit) {
+                        mbar_wait_bounded(&sm.a_full[h][s], par, a.err);
+                    } else {
+                        mbar_wait_bounded(&sm.a_full[0][s], par, a.err);
+                        mbar_wait_bounded(&sm.a_full[1][s], par, a.err);
+                    }
                     mbar_wait_bounded(&sm.full[s], par, a.err);
                     tc_fence_after();
                     // B stage: two 64-input halves of R token rows each (R = 64 or 128)
@@ -276,10 +311,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t bdesc0 = smem_desc_sw128(smem_u32(sm.b[s]));
                     const uint64_t bdesc1 = smem_desc_sw128(smem_u32(sm.b[s] + R * 128));
                     const uint32_t a_tmem = tmem + kACol0 + s * kAStageCols;
-#pragma unroll
-                    for (int j = 0; j < kBK / 16; ++j)
+                    for (int j = j0; j < j1; ++j)
                         tc_mma_ts(d_tmem, a_tmem + 8 * j, (j < 4 ? bdesc0 : bdesc1) + 2 * (j & 3), idesc,
-                                  (kc | j) != 0);
+                                  (kc | (j - j0)) != 0);
                     tc_commit(&sm.mma_done[s]);
                     if (++s == kStages) {
                         s = 0;
@@ -298,13 +332,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t it = 0, lt = 0, bph = 0;
         int bst = 0;   // ring stage of chunk it and its phase
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
-            const Tile tl = decode_tile(a, gateup, sm.pre, sm.off, t);
+            const Tile tl = decode_tile(a, gateup, nt, sm.pre, sm.off, t);
             if (!gateup) {
                 const int slot = lt % kTabs;
                 if (lt >= kTabs) mbar_wait_bounded(&sm.tab_empty[slot], ((lt / kTabs) - 1) & 1, a.err);
 #pragma unroll
-                for (int h = 0; h < kNT / 64; ++h) {   // 64 builder threads, kNT columns
+                for (int h = 0; h < kNTWide / 64; ++h) {   // 64 builder threads, nt columns
                     const int c = bt + 64 * h;
+                    if (c >= nt) break;
                     int tok = 0;
                     float w = 0.0f;
                     if (c < tl.nr) {
@@ -366,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t it = 0, lt = 0, dph = 0;
         int dst = 0;   // ring stage of chunk it and its phase
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
-            const Tile tl = decode_tile(a, gateup, sm.pre, sm.off, t);
+            const Tile tl = decode_tile(a, gateup, nt, sm.pre, sm.off, t);
             const int wrow = gateup ? ((L & 1) ? wrow_up(a, tl) : wrow_gate(a, tl)) + (L >> 1) : wrow_down(a, tl) + L;
             const uint32_t* sbrow = sbase + (size_t)wrow * ngroups;
             const int buf = lt & 1;
@@ -422,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.a_full[s]);
+                if (lane == 0) mbar_arrive(&sm.a_full[khalf][s]);
             }
             if (sb_tma) {
                 __syncwarp();
@@ -434,17 +469,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q = warp & 3;
         uint32_t lt = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
-            const Tile tl = decode_tile(a, gateup, sm.pre, sm.off, t);
-            const int ab = lt & 1;
+            const Tile tl = decode_tile(a, gateup, nt, sm.pre, sm.off, t);
             const int slot = lt % kTabs;
             if (!gateup) mbar_wait_bounded(&sm.tab_full[slot], (lt / kTabs) & 1, a.err);
+            const int ab = lt & 1;
             mbar_wait_bounded(&sm.acc_full[ab], (lt >> 1) & 1, a.err);
             tc_fence_after();
-            const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + ab * kNT;
+            const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (ksplit ? 2 : 1) * ab * nt;
             for (int c0 = 0; c0 < tl.npad; c0 += 16) {
+                // the sum of the two K-half accumulators (the warp is converged for
+                // the warp-wide tensor-memory loads)
                 uint32_t v[16];
+                __syncwarp();
                 tmem_ld16(taddr + c0, v);
-                tmem_ld_wait();
+                if (ksplit) {
+                    uint32_t v1[16];
+                    tmem_ld16(taddr + nt + c0, v1);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) v[c] = __float_as_uint(__uint_as_float(v[c]) + __uint_as_float(v1[c]));
+                } else {
+                    tmem_ld_wait();
+                }
                 if (gateup) {
                     // lanes 2i / 2i+1 hold gate / up of row j = 64 mb + 16 q + i; the
                     // even lane finishes the even columns, the odd lane the odd ones
@@ -646,6 +692,10 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     TcArgs ta;
     ta.f = a;
     ta.gateup = 1;
+    // narrow tiles on two MMA issuers when the experts hold few rows each
+    // (a tcgen05.mma stream costs about the same per instruction for any N)
+    ta.ksplit = (int64_t)a.T * a.K <= (int64_t)96 * a.E ? 1 : 0;
+    ta.nt = ta.ksplit ? kNTSplit : kNTWide;
     k_ffn_tc<<<G, kThreads, smem, st>>>(gu_map, x_map, x_map128, gsb_map, ta);
     ce = cudaGetLastError();
     if (ce != cudaSuccess) return ce;
