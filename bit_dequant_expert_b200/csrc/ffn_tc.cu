@@ -286,7 +286,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the two accumulators.
         const int h = warp == 1 ? 0 : 1;
         // one issuer (warp 1) for the whole chunk when the K halves are not split
-        const int j0 = ksplit ? 4 * h : 0, j1 = ksplit ? 4 * h + 4 : 8;
         if (lane == 0 && (ksplit || h == 0)) {
             uint32_t lt = 0, par = 0;
             int s = 0;   // ring stage and its phase, advanced per chunk
@@ -311,9 +310,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t bdesc0 = smem_desc_sw128(smem_u32(sm.b[s]));
                     const uint64_t bdesc1 = smem_desc_sw128(smem_u32(sm.b[s] + R * 128));
                     const uint32_t a_tmem = tmem + kACol0 + s * kAStageCols;
-                    for (int j = j0; j < j1; ++j)
-                        tc_mma_ts(d_tmem, a_tmem + 8 * j, (j < 4 ? bdesc0 : bdesc1) + 2 * (j & 3), idesc,
-                                  (kc | (j - j0)) != 0);
+                    // straight-line issue: a branch between two tcgen05.mma costs about
+                    // as much as the instruction itself
+                    if (ksplit) {
+                        const uint64_t bd = h ? bdesc1 : bdesc0;
+                        const uint32_t at = a_tmem + 32 * h;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) tc_mma_ts(d_tmem, at + 8 * j, bd + 2 * j, idesc, (kc | j) != 0);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            tc_mma_ts(d_tmem, a_tmem + 8 * j, (j < 4 ? bdesc0 : bdesc1) + 2 * (j & 3), idesc,
+                                      (kc | j) != 0);
+                    }
                     tc_commit(&sm.mma_done[s]);
                     if (++s == kStages) {
                         s = 0;
