@@ -50,6 +50,10 @@ namespace {
 constexpr int kWarps = 16;                      // compute warps
 constexpr int kThreads = (kWarps + 1) * 32;     // + one producer warp
 constexpr int kMaxT = 8;
+// Copies of the tagged router logits: every CTA polls all of a token's logits,
+// and 148 CTAs reading one 2 KB block at once queue on the L2 slices that hold
+// it; CTA b reads copy b mod kLogitCopies.
+constexpr int kLogitCopies = 8;
 constexpr int kJ = 32;                          // intermediate columns per unit
 constexpr int kMaxGuSlots = 6;                  // gate/up box ring (fewer when x needs the room)
 constexpr int kDnSlots = 2;                     // down ring: one unit's down columns each
@@ -120,7 +124,7 @@ struct DecArgs {
     FfnArgs f;
     DecLayout L;
     unsigned long long* launches;   // CTAs of decode launches so far (workspace header)
-    unsigned long long* tlogits;    // [kMaxT][E] tagged router logits (fused layer)
+    unsigned long long* tlogits;    // [kLogitCopies][kMaxT][E] tagged router logits (fused layer)
     DecodeRoute r;                  // fused layer: router inputs and routing outputs
     int lgI;                        // log2 of the intermediate size
 };
@@ -550,9 +554,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
 #pragma unroll
                     for (int off = 16; off >= 1; off >>= 1) accl = __fadd_rn(accl, __shfl_xor_sync(0xFFFFFFFFu, accl, off));
-                    if (lane == 0) {
+                    if (lane < kLogitCopies) {   // every lane holds the sum; one copy each
                         if (da.r.bias) accl = __fadd_rn(accl, da.r.bias[(int64_t)t * da.r.bias_stride + r_e]);
-                        st_relaxed_u64(da.tlogits + (size_t)t * E + r_e, tag_word(ep, accl));
+                        st_relaxed_u64(da.tlogits + (size_t)lane * kMaxT * E + (size_t)t * E + r_e, tag_word(ep, accl));
                     }
                 }
             }
@@ -570,7 +574,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     bool ok = true;
                     unsigned long long w[8];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) w[i] = ldcg_u64(da.tlogits + (size_t)warp * E + lane + 32 * i);
+                    for (int i = 0; i < 8; ++i)
+                        w[i] = ldcg_u64(da.tlogits + (size_t)(b % kLogitCopies) * kMaxT * E + (size_t)warp * E + lane + 32 * i);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         ok &= (uint32_t)w[i] == ep;
@@ -915,7 +920,7 @@ bool ffn_decode_supported(const FfnArgs& a) {
 size_t decode_ws_bytes(int T, int E, int I) {
     (void)T;
     (void)I;
-    return align256((size_t)kMaxT * E * 8);
+    return align256((size_t)kLogitCopies * kMaxT * E * 8);
 }
 
 DecodeWs decode_ws_carve(uint8_t* base, int T, int E, int I, unsigned long long* launches) {

@@ -102,7 +102,7 @@ cudaError_t launch_ffn_simt(const FfnArgs& a, cudaStream_t st);
 cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st);
 
 // Workspace sections of the decode kernels (T <= 8): the launch counter in
-// the workspace header and the tagged router logits.
+// the workspace header and the tagged router logits (several copies).
 struct DecodeWs {
     unsigned long long* launches;
     unsigned long long* tlogits;
