@@ -95,7 +95,7 @@ __device__ __forceinline__ void store_chunk(GdnSmem& sm, int buf, const ChunkReg
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 4) k_gdn_scan(GdnArgs a) {
+__global__ void __launch_bounds__(kThreads, 5) k_gdn_scan(GdnArgs a) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     GdnSmem& sm = *reinterpret_cast<GdnSmem*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
