@@ -200,6 +200,145 @@ __global__ void __launch_bounds__(kThreads, 5) k_gdn_scan(GdnArgs a) {
             make_float4(S[4 * m], S[4 * m + 1], S[4 * m + 2], S[4 * m + 3]);
 }
 
+// A handful of tokens (T <= kChunk: decode, verification): the call is a
+// stream of state rows (8 KB in, 8 KB out per 16 rows) with little
+// arithmetic between, so a resident CTA walks over several (sequence, head,
+// row block) items and fetches the next item's state (cp.async, 16 bytes a
+// copy) and inputs while it runs the current one.
+__device__ __forceinline__ void cp_async16(uint32_t dst_saddr, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_saddr), "l"(src) : "memory");
+}
+
+struct GdnSmallSmem {
+    GdnSmem base;               // k, q, v, decays, betas (two items), o
+    float s[2][kRows][kD];      // the state rows of the current and the next item
+};
+
+__global__ void __launch_bounds__(kThreads, 4) k_gdn_scan_small(GdnArgs a, int nitems) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    GdnSmallSmem& ss = *reinterpret_cast<GdnSmallSmem*>(smem_raw);
+    GdnSmem& sm = ss.base;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int lr = 4 * warp + (lane >> 3);   // the group's row within the item
+    const int c8 = lane & 7;                 // columns 32 m + 4 c8 + e
+    const int blocks_per_head = kD / kRows;
+    griddep_launch_dependents();
+    griddep_wait();   // the inputs and the state may come from the previous grid
+
+    struct Item {
+        int b, h, hk, row0;
+    };
+    auto coords = [&](int item) {
+        Item it;
+        const int bh = item / blocks_per_head;
+        it.h = bh % a.Hv;
+        it.b = bh / a.Hv;
+        it.hk = it.h / (a.Hv / a.Hk);
+        it.row0 = (item % blocks_per_head) * kRows;
+        return it;
+    };
+    auto fetch_state = [&](const Item& it, int sb) {
+        const float* src = a.state_in + ((size_t)(it.b * a.Hv + it.h) * kD + it.row0) * kD;
+        for (int p = tid; p < kRows * kD / 4; p += kThreads) cp_async16(smem_u32(&ss.s[sb][0][0] + 4 * p), src + 4 * p);
+        cp_async_commit();
+    };
+
+    int item = blockIdx.x;
+    if (item >= nitems) return;
+    ChunkRegs regs;
+    {
+        const Item it = coords(item);
+        fetch_state(it, 0);
+        load_chunk(a, it.b, it.h, it.hk, it.row0, 0, regs);
+    }
+    for (int n = 0; item < nitems; ++n) {
+        const int cur = n & 1;
+        const Item it = coords(item);
+        store_chunk(sm, cur, regs);
+        const int next = item + gridDim.x;
+        if (next < nitems) {
+            const Item nx = coords(next);
+            fetch_state(nx, cur ^ 1);
+            load_chunk(a, nx.b, nx.h, nx.hk, nx.row0, 0, regs);   // lands while this item runs
+            cp_async_wait<1>();   // this item's state (the older group) has landed
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+
+        float S[16];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const float4 v4 = *reinterpret_cast<const float4*>(&ss.s[cur][lr][32 * m + 4 * c8]);
+            S[4 * m] = v4.x;
+            S[4 * m + 1] = v4.y;
+            S[4 * m + 2] = v4.z;
+            S[4 * m + 3] = v4.w;
+        }
+        for (int st = 0; st < a.T; ++st) {
+            const float* kr = &sm.k[cur][st][4 * c8];
+            const float* qr = &sm.q[cur][st][4 * c8];
+            float kv[16];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const float4 v4 = *reinterpret_cast<const float4*>(kr + 32 * m);
+                kv[4 * m] = v4.x;
+                kv[4 * m + 1] = v4.y;
+                kv[4 * m + 2] = v4.z;
+                kv[4 * m + 3] = v4.w;
+            }
+            float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                p0 = fmaf(S[4 * m], kv[4 * m], p0);
+                p1 = fmaf(S[4 * m + 1], kv[4 * m + 1], p1);
+                p2 = fmaf(S[4 * m + 2], kv[4 * m + 2], p2);
+                p3 = fmaf(S[4 * m + 3], kv[4 * m + 3], p3);
+            }
+            float u = (p0 + p1) + (p2 + p3);
+            u += __shfl_xor_sync(0xFFFFFFFFu, u, 1);
+            u += __shfl_xor_sync(0xFFFFFFFFu, u, 2);
+            u += __shfl_xor_sync(0xFFFFFFFFu, u, 4);
+            const float dec = sm.a[cur][st];
+            const float w = sm.beta[cur][st] * (sm.v[cur][st][lr] - dec * u);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) S[j] = fmaf(dec, S[j], w * kv[j]);
+            float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const float4 q4 = *reinterpret_cast<const float4*>(qr + 32 * m);
+                r0 = fmaf(S[4 * m], q4.x, r0);
+                r1 = fmaf(S[4 * m + 1], q4.y, r1);
+                r2 = fmaf(S[4 * m + 2], q4.z, r2);
+                r3 = fmaf(S[4 * m + 3], q4.w, r3);
+            }
+            float o = (r0 + r1) + (r2 + r3);
+            o += __shfl_xor_sync(0xFFFFFFFFu, o, 1);
+            o += __shfl_xor_sync(0xFFFFFFFFu, o, 2);
+            o += __shfl_xor_sync(0xFFFFFFFFu, o, 4);
+            if (c8 == 0) sm.o[st][lr] = a.scale * o;
+        }
+        float* s_out = a.state_out + ((size_t)(it.b * a.Hv + it.h) * kD + it.row0 + lr) * kD;
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+            *reinterpret_cast<float4*>(s_out + 32 * m + 4 * c8) =
+                make_float4(S[4 * m], S[4 * m + 1], S[4 * m + 2], S[4 * m + 3]);
+        __syncthreads();   // o of the item complete
+        if (tid < 2 * a.T) {
+            const int st = tid >> 1, half = tid & 1;
+            const float* src = &sm.o[st][8 * half];
+            uint4 w4;
+            w4.x = pack_bf16x2(src[0], src[1]);
+            w4.y = pack_bf16x2(src[2], src[3]);
+            w4.z = pack_bf16x2(src[4], src[5]);
+            w4.w = pack_bf16x2(src[6], src[7]);
+            *reinterpret_cast<uint4*>(a.o + ((size_t)(it.b * a.T + st) * a.Hv + it.h) * kD + it.row0 + 8 * half) = w4;
+        }
+        __syncthreads();   // this item's buffers are free for the item after next
+        item = next;
+    }
+}
+
 }  // namespace
 
 bool gdn_scan_supported(const GdnArgs& a) {
@@ -208,6 +347,19 @@ bool gdn_scan_supported(const GdnArgs& a) {
 }
 
 cudaError_t launch_gdn_scan(const GdnArgs& a, cudaStream_t st) {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                   cudaSuccess)
+        return cudaErrorInvalidDevice;
+    const int nitems = a.B * a.Hv * (kD / kRows);
+    // the item-walking kernel pays off once every resident CTA gets two items or more
+    if (a.T <= kChunk && nitems >= 8 * sms) {
+        static int done_s[64] = {0};
+        const int smem_s = (int)sizeof(GdnSmallSmem);
+        cudaError_t ce = set_smem_once(k_gdn_scan_small, smem_s, done_s);
+        if (ce != cudaSuccess) return ce;
+        return launch_pdl(k_gdn_scan_small, dim3(4 * sms), dim3(kThreads), (size_t)smem_s, st, a, nitems);
+    }
     static int done[64] = {0};
     const int smem = (int)sizeof(GdnSmem);
     cudaError_t ce = set_smem_once(k_gdn_scan, smem, done);

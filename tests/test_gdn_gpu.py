@@ -57,6 +57,7 @@ def _check(d, o, S):
     (0, None, None),          # tiny, T = 17: one whole chunk of 16 tokens and a ragged tail
     (0, 1, 1), (0, 3, 16), (0, 2, 33),
     (1, 8, 1),                # decode: 8 sequences, one token, 16 key / 32 value heads
+    (1, 8, 4), (1, 5, 16),    # enough (sequence, head, row block) items for the item-walking kernel
     (2, None, None),          # verification: one sequence, 4 tokens
     (3, None, None),          # prefill: one sequence of 2048 tokens
 ])
@@ -103,4 +104,12 @@ def test_gdn_scan_edge_values():
     d["g"] = np.zeros_like(d["g"])
     o, S = _run(d)
     assert np.array_equal(S, d["S0"].astype(np.float64))
+    _check(d, o, S)
+
+
+def test_gdn_scan_item_walk_in_place():
+    """Decode shape (every CTA walks several items, prefetching the next
+    one's state): state_out may be state_in."""
+    d = gen.make_scan(gen.scan_config(1).with_B(7).with_T(2))
+    o, S = _run(d, in_place=True)
     _check(d, o, S)
