@@ -133,6 +133,8 @@ __global__ void __launch_bounds__(kThreads, 5) k_gdn_scan(GdnArgs a) {
         const int t0 = c * kChunk;
         if (c + 1 < nchunks) load_chunk(a, b, h, hk, row0, t0 + kChunk, regs);   // lands during the steps
         const int steps = min(kChunk, a.T - t0);
+        // two tokens per trip: a token's output reduction overlaps the next one's update
+#pragma unroll 2
         for (int s = 0; s < steps; ++s) {
             const float* kr = &sm.k[buf][s][4 * c8];
             const float* qr = &sm.q[buf][s][4 * c8];
