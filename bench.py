@@ -739,6 +739,18 @@ def run_ncu_case(case, device, calls):
 DECODE_WORKLOAD = "decode: T=1 x 40 distinct layers cycled (H 2048, I 512, E 256 top-8 + shared, G 64)"
 
 
+def decode_config(world: int) -> dict:
+    """The decode workload's config (the same for both arms)."""
+    return {
+        "workload": DECODE_WORKLOAD,
+        "global_batch": world,
+        "seq_len": 1,
+        "parallelism": "replicas" if world > 1 else "single GPU",
+        "l2": "inputs larger than L2 (18.2 GB of weights streamed per step; no flush)",
+        "graph": "one CUDA graph per step (40 layers x moe_decode_layer: decode kernel + combine)",
+    }
+
+
 def decode_line(res: dict, ms: float, units: float, world: int, steps: int, warmup: int, peaks: dict) -> dict:
     """The JSON line of the decode measurement: `ms` is the slowest rank's
     time per step, `units` the layer passes all ranks made per step, `res`
@@ -756,14 +768,7 @@ def decode_line(res: dict, ms: float, units: float, world: int, steps: int, warm
         "vs_baseline": None,
         "dtype": "bf16 (4-bit weights, fp32 accumulation)",
         "data": "synthetic (seeded; SplitMix64 layers shaped like the pages' model)",
-        "config": {
-            "workload": DECODE_WORKLOAD,
-            "global_batch": world,
-            "seq_len": 1,
-            "parallelism": "replicas" if world > 1 else "single GPU",
-            "l2": "inputs larger than L2 (18.2 GB of weights streamed per step; no flush)",
-            "graph": "one CUDA graph per step (40 layers x moe_decode_layer: decode kernel + combine)",
-        },
+        "config": decode_config(world),
         "decode_token_per_s": world / (ms / 1e3),
         "breakdown_us_per_layer": res["breakdown_us_per_layer"],
         "gpu_launches": res["gpu_launches"],
@@ -930,7 +935,7 @@ def run_reference(args, world, rank, warmup):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": len(per_step),
         "warmup": warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic (seeded)",
-        "config": {"workload": DECODE_WORKLOAD, "global_batch": 1, "seq_len": 1, "parallelism": "host cores"},
+        "config": decode_config(world),
         "impl": "reference",
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": omp_threads(), "cpu": cpu_model(), "kind": "oracle",
                          "sample": "one layer pass (T=1) per step, layers 0-2 cycled"},
