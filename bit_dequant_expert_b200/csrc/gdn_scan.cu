@@ -23,6 +23,7 @@
 #include "../../include/gdn_b200.h"
 #include "common.cuh"
 #include "kernels.h"
+#include "api_range.h"
 #include "ptx.cuh"
 
 namespace moe {
@@ -382,6 +383,7 @@ bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0
 extern "C" int32_t gdn_scan(int32_t B, int32_t T, int32_t Hk, int32_t Hv, int32_t dk, int32_t dv, const uint16_t* q,
                             const uint16_t* k, const uint16_t* v, const float* g, const float* beta, float scale,
                             const float* state_in, float* state_out, uint16_t* o, void* stream) {
+    moe::ApiRange api_range("gdn_scan");
     if (B < 1 || T < 1 || Hk < 1 || Hv < 1) return MOE_ERR_INVALID_ARG;
     if (!q || !k || !v || !g || !beta || !state_in || !state_out || !o) return MOE_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state_in) || !aligned16(state_out) ||

@@ -4,6 +4,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "api_range.h"
 
 using namespace moe;
 
@@ -98,6 +99,7 @@ size_t moe_workspace_size(const moe_config_t* cfg, int32_t max_tokens) {
 }
 
 int32_t moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+    moe::ApiRange api_range("moe_workspace_init");
     if (!ws || ws_bytes < sizeof(WsHeader) || !aligned(ws, 256)) return MOE_ERR_WORKSPACE;
     // all of it: the decode kernels' tagged words must not match a restarted launch count
     return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream));
@@ -106,6 +108,7 @@ int32_t moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
 int32_t moe_route(const moe_config_t* cfg, int32_t T, const uint16_t* x, const uint16_t* w_router,
                   const float* logits_in, const float* logit_bias, int64_t logit_bias_row_stride,
                   int32_t* topk_idx, float* topk_w, int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
+    moe::ApiRange api_range("moe_route");
     if (!ws) return MOE_ERR_WORKSPACE;
     int32_t st = check_common(cfg, T, ws, ws_bytes);
     if (st) return st;
@@ -137,6 +140,7 @@ int32_t moe_route(const moe_config_t* cfg, int32_t T, const uint16_t* x, const u
 int32_t moe_router_logits(const moe_config_t* cfg, int32_t T, const uint16_t* x, const uint16_t* w_router,
                           const float* logit_bias, int64_t logit_bias_row_stride, float* logits, void* ws,
                           size_t ws_bytes, void* stream) {
+    moe::ApiRange api_range("moe_router_logits");
     if (!ws) return MOE_ERR_WORKSPACE;
     int32_t st = check_common(cfg, T, ws, ws_bytes);
     if (st) return st;
@@ -161,6 +165,7 @@ int32_t moe_router_logits(const moe_config_t* cfg, int32_t T, const uint16_t* x,
 int32_t moe_permute(const moe_config_t* cfg, int32_t T, const int32_t* topk_idx, const int32_t* counts,
                     int32_t* offsets, int32_t* row_to_pair, int32_t* pair_to_row, void* ws, size_t ws_bytes,
                     void* stream) {
+    moe::ApiRange api_range("moe_permute");
     if (!ws) return MOE_ERR_WORKSPACE;
     int32_t st = check_common(cfg, T, ws, ws_bytes);
     if (st) return st;
@@ -187,6 +192,7 @@ int32_t moe_expert_ffn_path(const moe_config_t* cfg, int32_t T, const uint16_t* 
                             const int32_t* offsets, const int32_t* row_to_pair, const float* topk_w,
                             int32_t mode, void* out0, void* out1, void* ws, size_t ws_bytes, int32_t path,
                             void* stream) {
+    moe::ApiRange api_range("moe_expert_ffn_path");
     if (!ws) return MOE_ERR_WORKSPACE;
     int32_t st = check_common(cfg, T, ws, ws_bytes);
     if (st) return st;
@@ -251,6 +257,7 @@ int32_t moe_expert_ffn(const moe_config_t* cfg, int32_t T, const uint16_t* x, co
 
 int32_t moe_combine(const moe_config_t* cfg, int32_t T, int32_t mode, const void* in0, const void* in1,
                     const int32_t* pair_to_row, const float* topk_w, uint16_t* y, void* stream) {
+    moe::ApiRange api_range("moe_combine");
     int32_t st = check_common(cfg, T, nullptr, 0);
     if (st) return st;
     if (mode != MOE_MODE_SCATTER && mode != MOE_MODE_PAIRS) return MOE_ERR_INVALID_ARG;
@@ -279,6 +286,7 @@ int32_t moe_combine(const moe_config_t* cfg, int32_t T, int32_t mode, const void
 int32_t moe_gather_rows(const moe_config_t* cfg, int32_t T, const uint16_t* x, const int32_t* row_to_pair,
                         const float* topk_w, int32_t row_begin, int32_t n_rows, uint16_t* rows_out, float* w_out,
                         void* ws, size_t ws_bytes, void* stream) {
+    moe::ApiRange api_range("moe_gather_rows");
     if (!ws) return MOE_ERR_WORKSPACE;
     int32_t st = check_common(cfg, T, ws, ws_bytes);
     if (st) return st;
@@ -319,6 +327,7 @@ int32_t moe_decode_layer(const moe_config_t* cfg, int32_t T, const uint16_t* x, 
                          float* topk_w, int32_t* counts, int32_t* offsets, int32_t* row_to_pair,
                          int32_t* pair_to_row, float* y_acc, uint16_t* y, void* ws, size_t ws_bytes,
                          void* stream) {
+    moe::ApiRange api_range("moe_decode_layer");
     if (!ws) return MOE_ERR_WORKSPACE;
     int32_t st = check_common(cfg, T, ws, ws_bytes);
     if (st) return st;

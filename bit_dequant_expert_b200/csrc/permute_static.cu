@@ -12,6 +12,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "api_range.h"
 
 namespace {
 
@@ -51,6 +52,7 @@ bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0
 extern "C" int32_t moe_permute_static(const moe_config_t* cfg, int32_t T, const int32_t* topk_idx,
                                       const int32_t* counts, int32_t* offsets, int32_t* row_to_pair,
                                       int32_t* pair_to_row, int32_t* err_out, void* stream) {
+    moe::ApiRange api_range("moe_permute_static");
     if (!cfg) return MOE_ERR_INVALID_ARG;
     if (cfg->num_experts != 256 || cfg->top_k != 8 || cfg->group_size != 64 || cfg->hidden < 256 ||
         cfg->hidden % 256 != 0 || cfg->inter < 128 || cfg->inter % 128 != 0 ||
