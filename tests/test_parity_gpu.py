@@ -164,7 +164,7 @@ def test_permute_rejects_bad_routing():
     assert m.moe_get_device_error(ws) == m.MOE_ERR_BOUNDS
 
 
-@pytest.mark.parametrize("T", [1, 100, 256, 257, 1000, 5000])
+@pytest.mark.parametrize("T", [1, 100, 256, 257, 1000, 4096, 4097, 5000])
 def test_permute_bitexact_random(T):
     import torch
     import bit_dequant_expert_b200 as m

@@ -72,7 +72,7 @@ def test_permute_static_changing_sizes_back_to_back():
         _check(m, cfg, _routing(T, seed))
 
 
-@pytest.mark.parametrize("T", [4, 5000])
+@pytest.mark.parametrize("T", [4, 1000, 5000])
 def test_permute_static_reports_bad_routing(T):
     """A repeated expert within a token, then an index out of range, come back
     as MOE_ERR_BOUNDS in err_out; a clean call afterwards reports MOE_OK."""
