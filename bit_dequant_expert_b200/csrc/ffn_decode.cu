@@ -163,6 +163,14 @@ __device__ __forceinline__ void sb_factor(uint32_t w, float& s, float& bp) {
     bp = fmaf(-128.0f, s, __uint_as_float(w & 0xFFFF0000u));
 }
 
+// Down-phase staging of a warp's 16-row tile, [token][row] floats in 16-float
+// slots: token t in slot (t odd) * 4 + t / 2, row quads of tokens 4..7 swapped
+// in pairs.  The four stores of a lane (rows g, g + 8; tokens 2c, 2c + 1) and
+// the 8-lane phases of the float4 reads each touch 32 distinct banks.
+__device__ __forceinline__ int stage_word(int t, int r) {
+    return 16 * ((t & 1) * 4 + (t >> 1)) + 4 * ((r >> 2) ^ (((t >> 2) & 1) << 1)) + (r & 3);
+}
+
 __device__ __forceinline__ uint2 lds64(const uint8_t* p) { return *reinterpret_cast<const uint2*>(p); }
 __device__ __forceinline__ uint32_t lds32(const uint8_t* p) { return *reinterpret_cast<const uint32_t*>(p); }
 
@@ -424,7 +432,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             zero_seen = true;
         }
         const bool two = T > 1;   // odd token columns hold tokens
-        const bool lead = (g & 3) == 0;
+        float* stg = reinterpret_cast<float*>(red) + warp * 128;   // this warp's staging area
+        // what this lane reduces: 16-float slot lane / 4 (token rd_t), its float4 lane % 4 (rows rd_row..+3)
+        const int rd_s = lane >> 2;
+        const int rd_t = rd_s < 4 ? 2 * rd_s : 2 * (rd_s - 4) + 1;
+        const int rd_row = 4 * ((lane & 3) ^ (((rd_t >> 2) & 1) << 1));
 #pragma unroll
         for (int tt = 0; tt < kTW; ++tt) {
             const int n = 16 * (warp + kWarps * tt) + g;
@@ -438,39 +450,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             // w (s D + (b - 128 s) sum(h)) for rows n (d0, d1) and n + 8 (d2, d3), tokens 2c, 2c+1
             const float v0 = w0 != 0.0f ? w0 * fmaf(sa, d[0], ba * hs0) : 0.0f;
             const float v2 = w0 != 0.0f ? w0 * fmaf(sb2, d[2], bb2 * hs0) : 0.0f;
-            // lanes g = 0, 4 gather rows g..g+3 of their column from lanes g+1..g+3: one vector reduction
-            float4 q0, q2;
-            q0.x = v0;
-            q0.y = __shfl_down_sync(0xFFFFFFFFu, v0, 4);
-            q0.z = __shfl_down_sync(0xFFFFFFFFu, v0, 8);
-            q0.w = __shfl_down_sync(0xFFFFFFFFu, v0, 12);
-            q2.x = v2;
-            q2.y = __shfl_down_sync(0xFFFFFFFFu, v2, 4);
-            q2.z = __shfl_down_sync(0xFFFFFFFFu, v2, 8);
-            q2.w = __shfl_down_sync(0xFFFFFFFFu, v2, 12);
-            if (lead && 2 * c < T) {
-                float* y0 = a.y_acc + (size_t)(2 * c) * kH + n;
-                red_add_v4(y0, q0.x, q0.y, q0.z, q0.w);
-                red_add_v4(y0 + 8, q2.x, q2.y, q2.z, q2.w);
-            }
-            if (two) {
-                const float v1 = w1 != 0.0f ? w1 * fmaf(sa, d[1], ba * hs1) : 0.0f;
-                const float v3 = w1 != 0.0f ? w1 * fmaf(sb2, d[3], bb2 * hs1) : 0.0f;
-                float4 q1, q3;
-                q1.x = v1;
-                q1.y = __shfl_down_sync(0xFFFFFFFFu, v1, 4);
-                q1.z = __shfl_down_sync(0xFFFFFFFFu, v1, 8);
-                q1.w = __shfl_down_sync(0xFFFFFFFFu, v1, 12);
-                q3.x = v3;
-                q3.y = __shfl_down_sync(0xFFFFFFFFu, v3, 4);
-                q3.z = __shfl_down_sync(0xFFFFFFFFu, v3, 8);
-                q3.w = __shfl_down_sync(0xFFFFFFFFu, v3, 12);
-                if (lead && 2 * c + 1 < T) {
-                    float* y1 = a.y_acc + (size_t)(2 * c + 1) * kH + n;
-                    red_add_v4(y1, q1.x, q1.y, q1.z, q1.w);
-                    red_add_v4(y1 + 8, q3.x, q3.y, q3.z, q3.w);
-                }
-            }
+            const float v1 = (two && w1 != 0.0f) ? w1 * fmaf(sa, d[1], ba * hs1) : 0.0f;
+            const float v3 = (two && w1 != 0.0f) ? w1 * fmaf(sb2, d[3], bb2 * hs1) : 0.0f;
+            // the tile's [8 tokens][16 rows] through the warp's staging area, then one vector
+            // reduction of 4 consecutive rows of one token per lane
+            stg[stage_word(2 * c, g)] = v0;
+            stg[stage_word(2 * c, g + 8)] = v2;
+            stg[stage_word(2 * c + 1, g)] = v1;
+            stg[stage_word(2 * c + 1, g + 8)] = v3;
+            __syncwarp();
+            const float4 r4 = *reinterpret_cast<const float4*>(stg + 16 * (lane >> 2) + 4 * (lane & 3));
+            if (rd_t < T) red_add_v4(a.y_acc + (size_t)rd_t * kH + 16 * (warp + kWarps * tt) + rd_row, r4.x, r4.y, r4.z, r4.w);
+            __syncwarp();   // the next tile overwrites the staging area
         }
         __syncwarp();
         if (lane == 0) {
