@@ -39,6 +39,7 @@ MOE_PATH_AUTO = 0
 MOE_PATH_SIMT = 1
 MOE_PATH_GEMV = 2
 MOE_PATH_TC = 3
+MOE_PATH_TC_GEMV = 4
 
 EXPORTED = (
     "moe_workspace_size", "moe_workspace_init", "moe_route", "moe_permute", "moe_expert_ffn",

@@ -60,7 +60,12 @@ constexpr int kDnSlots = 2;                     // down ring: one unit's down co
 constexpr int kMaxSlots = 1 + 8 * kMaxT;        // active experts: shared + 8 per token
 constexpr int kSmemLimit = 232448;              // dynamic shared memory per block (227 KB)
 constexpr int kRouterRows = 2;                  // router rows per CTA (experts b and b + grid size)
-constexpr int kExtraBars = 7;                   // mbarriers besides the two rings
+constexpr int kExtraBars = 9;                   // mbarriers besides the two rings
+constexpr int kMaxRows = 8;                     // row-list launches: experts of at most this many rows
+// k_decode modes: the T <= 8 tokens of a launch (four-call path), the same
+// with the routing fused in, or the rows of the experts that hold few of them
+// (the tensor-core path's small experts)
+constexpr int kModeTokens = 0, kModeRoute = 1, kModeRows = 2;
 
 struct DecLayout {
     int gu_box;     // gate/up codes box: 16 rows x H/2 bytes
@@ -75,10 +80,10 @@ struct DecLayout {
 
 // Routing state of the CTA (shared memory).
 struct DecTab {
-    int slot_e[kMaxSlots + 7];          // expert of each active slot (slot 0 = shared when present)
+    int slot_e[256 + 8];                // expert of each active slot (slot 0 = shared when present)
     float wsel[kMaxSlots + 7][kMaxT];   // routing weight of (slot, token); 0 = not routed there
     int slot_of[256];                   // active slot of each expert
-    int off[260];                       // expert offsets (routing outputs)
+    int off[260];                       // expert offsets (routing outputs; the row list of a row-list launch)
     int sel[8 * kMaxT];                 // selected expert per pair (fused layer)
     float selw[8 * kMaxT];              // its weight
     float hsum[2][4][kMaxT];            // per unit parity and box: sums of the rounded h per token
@@ -90,6 +95,10 @@ struct DecTab {
 };
 
 __host__ __device__ inline int round_up(int v, int a) { return (v + a - 1) / a * a; }
+
+// Row-list launch: units a CTA can hold the column tables of (token, weight per
+// column: 8 bytes x kMaxRows), in the router-row area the other modes use.
+__host__ __device__ constexpr int row_units_cap(int H) { return kRouterRows * 2 * H / (8 * kMaxRows); }
 
 DecLayout dec_layout(int H, int I, int T) {
     DecLayout L;
@@ -178,7 +187,7 @@ __device__ __forceinline__ unsigned long long tag_word(uint32_t epoch, float v) 
     return ((unsigned long long)__float_as_uint(v) << 32) | epoch;
 }
 
-template <int kH, bool kRoute>
+template <int kH, int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     k_decode(const __grid_constant__ CUtensorMap gu_map, const __grid_constant__ CUtensorMap gsb_map,
              const __grid_constant__ CUtensorMap dn_map, const __grid_constant__ CUtensorMap dsb_map,
@@ -191,6 +200,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kXS = 2 * kH + 16;             // x row stride in shared memory (bytes)
     constexpr int kRChunks = kH / 256;           // router chunks per lane
     constexpr int kTW = kH / 256;                // 16-row down tiles per warp
+    constexpr bool kRoute = kMode == kModeRoute;
+    constexpr bool kRows = kMode == kModeRows;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const FfnArgs& a = da.f;
@@ -202,7 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int g = lane >> 2, c = lane & 3;
     const int rg = perm8(g);
     const int NJ = I >> 5;                       // units per expert
-    const bool sh = a.has_shared != 0;
+    const bool sh = !kRows && a.has_shared != 0;   // a row-list launch leaves the shared expert to its caller
     const bool early_unit = sh && b < NJ;        // the first unit is the shared expert's block b
     const int gus = L.gu_slots;
 
@@ -219,11 +230,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* zeroed = rt_full + 4;       // this CTA's slice of y_acc is cleared (producer lane 0 waits)
     uint64_t* dsb_full = rt_full + 5;     // the unit's down (scale, bias) box landed (TMA form)
     uint64_t* dsb_empty = rt_full + 6;    // and was read by every compute warp
+    uint64_t* x_full = rt_full + 7;       // row-list launch: the unit's x rows landed
+    uint64_t* x_empty = rt_full + 8;      // and were read by every compute warp
     uint8_t* xs = smem + L.off_x;                                    // [T][kH] bf16, split order
     float* sx = reinterpret_cast<float*>(smem + L.off_sx);           // [kNG][kMaxT] group sums of x
     float4* red = reinterpret_cast<float4*>(smem + L.off_red);       // [kWarps][32]
     uint16_t* hs = reinterpret_cast<uint16_t*>(smem + L.off_hs);     // [2][kMaxT][kJ] h of a unit, split order
     uint32_t* dsb = reinterpret_cast<uint32_t*>(smem + L.off_dsb);   // [kH] down (scale, bias) words of a unit
+    // row-list launch: token and routing weight of each column of this CTA's units (router-row area)
+    int* utok = reinterpret_cast<int*>(smem + L.off_rt);                         // [unit][kMaxRows]
+    float* uw = reinterpret_cast<float*>(smem + L.off_rt) + row_units_cap(kH) * kMaxRows;
 
     if (tid == 0) {
         for (int i = 0; i < gus; ++i) {
@@ -241,6 +257,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(zeroed, 1);
         mbar_init(dsb_full, 1);
         mbar_init(dsb_empty, kWarps);
+        mbar_init(x_full, 1);
+        mbar_init(x_empty, 1);
         fence_mbar_init();
     }
     if (warp == kWarps && lane == 0) {
@@ -253,11 +271,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- loads (producer lane 0)
     // gate/up boxes of a unit (expert e, column block jb), then its down columns
-    int gu_n = 0, gu_cs = 0, gu_ph = 0, dn_n = 0, sb_n = 0;
+    int gu_n = 0, gu_cs = 0, gu_ph = 0, dn_n = 0, sb_n = 0, x_n = 0;
     // Producer lane 0: the first reductions into y_acc wait until every CTA has
     // cleared its slice.  release_zero polls the launch counter for that and
     // opens zero_done; it must run before any load waits on a down phase.
-    bool released = false;
+    bool released = kRows;   // a row-list launch adds into y_acc as it is
     auto release_zero = [&]() {
         const unsigned long long target = tab.zero_target;
         const uint64_t t0 = globaltimer_ns();
@@ -273,6 +291,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         released = true;
     };
     auto issue_unit = [&](int e, int jb) {
+        if (kRows) {
+            // the expert's gathered x rows (split order, rows off[e].. of xg) into the one x slot,
+            // once the previous unit's gate/up has read it
+            if (x_n >= 1) mbar_wait_bounded(x_empty, (x_n - 1) & 1, a.err);
+            const int lo = tab.off[e], n = min(max(tab.slot_of[e], 0), kMaxRows);   // slot_of: rows of each expert
+            mbar_arrive_expect_tx(x_full, (uint32_t)(n * 2 * kH));
+            for (int r = 0; r < n; ++r)
+                bulk_load(xs + (size_t)r * kXS, a.xg + (size_t)(lo + r) * kH, 2 * kH, x_full);
+            ++x_n;
+        }
         for (int p = 0; p < 4; ++p) {
             if (gu_n >= gus) mbar_wait_bounded(&gu_empty[gu_cs], (gu_ph - 1) & 1, a.err);
             mbar_arrive_expect_tx(&gu_full[gu_cs], L.gu_box + kH);
@@ -325,8 +353,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the same up row) and K quarter kq = w >> 2.  Down: warp w takes the 16-row
     // tiles w, w + 16, ... of all H rows, K = the unit's 32 columns.
     const int p_box = warp & 3, kq = warp >> 2;
-    const int gt = g < T ? g : T - 1;            // absent tokens read a present one; their weight is 0
-    const uint8_t* xrow = xs + (size_t)gt * kXS + 32 * c;
+    const int gt_all = g < T ? g : T - 1;        // absent tokens read a present one; their weight is 0
+    int* rows_n = tab.slot_of;                   // row-list launch: rows of each expert (a route-mode table otherwise)
+    // group sums of x, per column: thread (gr, t)
+    auto x_group_sums = [&](int ncols) {
+        if (tid < kNG * kMaxT) {
+            const int gr = tid >> 3, t = tid & 7;
+            float sum = 0.0f;
+            if (t < ncols) {
+                const uint4* px = reinterpret_cast<const uint4*>(xs + (size_t)t * kXS + 128 * gr);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const uint4 v = px[u];
+                    sum += (bf16_lo(v.x) + bf16_hi(v.x)) + (bf16_lo(v.y) + bf16_hi(v.y)) +
+                           (bf16_lo(v.z) + bf16_hi(v.z)) + (bf16_lo(v.w) + bf16_hi(v.w));
+                }
+            }
+            sx[gr * kMaxT + t] = sum;
+        }
+    };
     auto code_off = [&](int gr) -> uint32_t {
         return (uint32_t)(((gr >> 2) * 8 + rg) * 128) + (((uint32_t)((2 * (gr & 3)) | (c >> 1)) ^ (uint32_t)rg) << 4) +
                (uint32_t)((c & 1) << 3);
@@ -336,9 +381,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         return o ^ (((o >> 7) & kSmask) << 4);
     };
     int cu_n = 0, cu_cs = 0, cu_ph = 0;   // consumers' view of the gate/up ring
-    bool zero_seen = false;
+    bool zero_seen = kRows;   // a row-list launch adds into y_acc as it is
     auto compute_unit = [&](int k, int s, int jb) {
         const int e = tab.slot_e[s];
+        // MMA columns holding tokens (row-list launch: the expert's rows); absent columns read a
+        // present one, and their weight is 0
+        const int ncol = kRows ? rows_n[e] : T;
+        const int gt = kRows ? (g < ncol ? g : ncol - 1) : gt_all;
+        const uint8_t* xrow = xs + (size_t)gt * kXS + 32 * c;
+        if (kRows) {
+            mbar_wait_bounded(x_full, k & 1, a.err);
+            x_group_sums(ncol);
+            named_barrier(1, kWarps * 32);
+        }
         // the down (scale, bias) word of every row for this block's group of I (the
         // TMA form lands with the unit's other boxes)
         if (!L.sb_tma) {
@@ -412,17 +467,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         cp_async_wait<0>();
         named_barrier(1, kWarps * 32);   // h, its sums and the down (scale, bias) words complete; red[] free
+        if (kRows && tid == 0) mbar_arrive(x_empty);   // x and its sums read
         // ---- down: rows 16 t + {g, g + 8} of tile t, K = the block's 32 columns
         const int ds = k & 1;
         mbar_wait_bounded(&dn_full[ds], (k >> 1) & 1, a.err);
         const uint8_t* dbox = smem + L.off_dn + ds * L.dn_box;   // [kH rows][4 words]
         const uint4 hv = *reinterpret_cast<const uint4*>(hk + gt * kJ + 8 * c);
-        const int t0c = 2 * c < T ? 2 * c : T - 1, t1c = 2 * c + 1 < T ? 2 * c + 1 : T - 1;
+        const int t0c = 2 * c < ncol ? 2 * c : ncol - 1, t1c = 2 * c + 1 < ncol ? 2 * c + 1 : ncol - 1;
         const float hs0 = (tab.hsum[k & 1][0][t0c] + tab.hsum[k & 1][1][t0c]) +
                           (tab.hsum[k & 1][2][t0c] + tab.hsum[k & 1][3][t0c]);
         const float hs1 = (tab.hsum[k & 1][0][t1c] + tab.hsum[k & 1][1][t1c]) +
                           (tab.hsum[k & 1][2][t1c] + tab.hsum[k & 1][3][t1c]);
-        const float w0 = tab.wsel[s][2 * c], w1 = tab.wsel[s][2 * c + 1];
+        const float* wcol = kRows ? uw + k * kMaxRows : tab.wsel[s];
+        const float w0 = wcol[2 * c], w1 = wcol[2 * c + 1];
         if (L.sb_tma) mbar_wait_bounded(dsb_full, k & 1, a.err);
         // row n's word: a 16-byte piece per row holding word (jb / 2) % 4 (TMA form), else one word per row
         const uint8_t* sbrow = reinterpret_cast<const uint8_t*>(dsb) + (L.sb_tma ? 4 * ((jb >> 1) & 3) : 0);
@@ -431,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait_bounded(zero_done, 0, a.err);
             zero_seen = true;
         }
-        const bool two = T > 1;   // odd token columns hold tokens
+        const bool two = ncol > 1;   // odd columns hold tokens
         float* stg = reinterpret_cast<float*>(red) + warp * 128;   // this warp's staging area
         // what this lane reduces: 16-float slot lane / 4 (token rd_t), its float4 lane % 4 (rows rd_row..+3)
         const int rd_s = lane >> 2;
@@ -460,7 +517,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             stg[stage_word(2 * c + 1, g + 8)] = v3;
             __syncwarp();
             const float4 r4 = *reinterpret_cast<const float4*>(stg + 16 * (lane >> 2) + 4 * (lane & 3));
-            if (rd_t < T) red_add_v4(a.y_acc + (size_t)rd_t * kH + 16 * (warp + kWarps * tt) + rd_row, r4.x, r4.y, r4.z, r4.w);
+            if (rd_t < ncol)
+                red_add_v4(a.y_acc + (size_t)(kRows ? utok[k * kMaxRows + rd_t] : rd_t) * kH + 16 * (warp + kWarps * tt) + rd_row,
+                           r4.x, r4.y, r4.z, r4.w);
             __syncwarp();   // the next tile overwrites the staging area
         }
         __syncwarp();
@@ -479,15 +538,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             lo = __ldcg(a.offsets + tid);
             hi = __ldcg(a.offsets + tid + 1);
         }
-        // this CTA's slice of y_acc
-        {
+        // this CTA's slice of y_acc (a row-list launch adds into it as it is)
+        if (!kRows) {
             const size_t n4 = (size_t)T * kH / 4, per = (n4 + G - 1) / G;
             const size_t lo4 = (size_t)b * per, hi4 = min(n4, lo4 + per);
             for (size_t q = lo4 + tid; q < hi4; q += kWarps * 32)
                 reinterpret_cast<float4*>(a.y_acc)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        // x (split order)
-        for (int t = 0; t < T; ++t) {
+        // x (split order; a row-list launch loads each unit's rows)
+        for (int t = 0; t < (kRows ? 0 : T); ++t) {
             for (int c8 = tid; c8 < kH / 8; c8 += kWarps * 32) {
                 const uint4 v = *reinterpret_cast<const uint4*>(a.x + (size_t)t * kH + 8 * c8);
                 *reinterpret_cast<uint4*>(xs + (size_t)t * kXS + 16 * c8) = to_split_order(v);
@@ -501,21 +560,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tab.slot_e[0] = E;
             mbar_arrive(zeroed);   // the slice is cleared; the producer counts this CTA
         }
-        // group sums of x, per token: thread (gr, t)
-        if (tid < kNG * kMaxT) {
-            const int gr = tid >> 3, t = tid & 7;
-            float s = 0.0f;
-            if (t < T) {
-                const uint4* px = reinterpret_cast<const uint4*>(xs + (size_t)t * kXS + 128 * gr);
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const uint4 v = px[u];
-                    s += (bf16_lo(v.x) + bf16_hi(v.x)) + (bf16_lo(v.y) + bf16_hi(v.y)) +
-                         (bf16_lo(v.z) + bf16_hi(v.z)) + (bf16_lo(v.w) + bf16_hi(v.w));
-                }
-            }
-            sx[gr * kMaxT + t] = s;
-        }
+        if (!kRows) x_group_sums(T);
         const int first = sh ? 1 : 0;
         if (kRoute) {
             // ---- router logits of this CTA's experts in the contract order: lane l
@@ -655,7 +700,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     set_error(a.err, MOE_ERR_BOUNDS);
                     lo = hi = 0;
                 }
-                act = hi > lo;
+                act = hi > lo && (!kRows || hi - lo <= kMaxRows);
+                if (kRows) {
+                    tab.off[tid] = lo;
+                    rows_n[tid] = hi - lo;
+                }
             }
             const uint32_t bal = __ballot_sync(0xFFFFFFFFu, act);
             if (lane == 0) tab.wtot[warp] = __popc(bal);
@@ -675,8 +724,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             named_barrier(1, kWarps * 32);
             if (tid == 0) mbar_arrive(list_ready);   // the active list is ready for the producer
+            if (kRows) {
+                // token and routing weight of each column of this CTA's units
+                const int nk = min(b < tab.A * NJ ? (tab.A * NJ - 1 - b) / G + 1 : 0, row_units_cap(kH));
+                for (int q = tid; q < nk * kMaxRows; q += kWarps * 32) {
+                    const int kk = q / kMaxRows, cc = q % kMaxRows;
+                    const int ee = tab.slot_e[(b + kk * G) >> (lgI - 5)];
+                    int tk = 0;
+                    float ww = 0.0f;
+                    if (cc < rows_n[ee]) {
+                        const int pr = __ldcg(a.row_to_pair + tab.off[ee] + cc);
+                        if (pr < 0 || pr >= T * a.K) {
+                            set_error(a.err, MOE_ERR_BOUNDS);
+                        } else {
+                            tk = pr / a.K;
+                            ww = __ldcg(a.topk_w + pr);
+                        }
+                    }
+                    utok[q] = tk;
+                    uw[q] = ww;
+                }
+            }
             // routing weights of each (slot, token)
-            if (act) {
+            if (!kRows && act) {
                 for (int r = lo; r < hi; ++r) {
                     const int p = __ldcg(a.row_to_pair + r);
                     if (p < 0 || p >= T * a.K) {
@@ -693,7 +763,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int A = tab.A;
         int k = 0, u = b, s = b >> (lgI - 5), jb = b & (NJ - 1);
         const int dsl = G >> (lgI - 5), dj = G & (NJ - 1);   // advance of (slot, block) per unit
-        for (; u < A * NJ; u += G, ++k) {
+        const int kcap = kRows ? row_units_cap(kH) : 1 << 30;   // units whose column tables fit
+        for (; u < A * NJ && k < kcap; u += G, ++k) {
             if (!(kRoute && k == 0 && early_unit)) compute_unit(k, s, jb);   // else done above
             s += dsl;
             jb += dj;
@@ -705,16 +776,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ---------------------------------------------------------- producer
         if (lane == 0) {
-            // the launch number, and the count at which every CTA has cleared its slice of y_acc
-            const unsigned long long v = ld_relaxed_u64(da.launches);
-            tab.epoch = (uint32_t)((v / (unsigned long long)G) % 0xFFFFFFFFull) + 1u;
-            tab.zero_target = (v / (unsigned long long)G + 1ull) * (unsigned long long)G;
-            mbar_arrive(zt_ready);
-            // count this CTA once its slice is cleared (the consumers' stores, seen through
-            // the mbarrier, are ordered before the count by the fence)
-            mbar_wait_bounded(zeroed, 0, a.err);
-            __threadfence();
-            red_add_relaxed_u64(da.launches, 1ull);
+            if (!kRows) {   // a row-list launch neither clears y_acc nor counts itself
+                // the launch number, and the count at which every CTA has cleared its slice of y_acc
+                const unsigned long long v = ld_relaxed_u64(da.launches);
+                tab.epoch = (uint32_t)((v / (unsigned long long)G) % 0xFFFFFFFFull) + 1u;
+                tab.zero_target = (v / (unsigned long long)G + 1ull) * (unsigned long long)G;
+                mbar_arrive(zt_ready);
+                // count this CTA once its slice is cleared (the consumers' stores, seen through
+                // the mbarrier, are ordered before the count by the fence)
+                mbar_wait_bounded(zeroed, 0, a.err);
+                __threadfence();
+                red_add_relaxed_u64(da.launches, 1ull);
+            }
             // the fused layer's shared-expert unit reduces into y_acc before the active
             // list exists; otherwise units 0 and 1 go first (their loads never wait on a
             // reduction), then the release, then the rest
@@ -723,7 +796,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int A = tab.A;
             int u = b, s = b >> (lgI - 5), jb = b & (NJ - 1), k = 0;
             const int dsl = G >> (lgI - 5), dj = G & (NJ - 1);
-            for (; u < A * NJ; u += G, ++k) {
+            const int kcap = kRows ? row_units_cap(kH) : 1 << 30;
+            for (; u < A * NJ && k < kcap; u += G, ++k) {
                 if (!released && k == 2) release_zero();
                 if (!(u == b && early_unit)) issue_unit(tab.slot_e[s], jb);
                 s += dsl;
@@ -834,17 +908,17 @@ bool make_dsb_map(CUtensorMap* m, const FfnArgs& a) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int kH, bool kRoute>
+template <int kH, int kMode>
 cudaError_t launch_dec_h(const DecArgs& da, const CUtensorMap& gu_map, const CUtensorMap& gsb_map,
                          const CUtensorMap& dn_map, const CUtensorMap& dsb_map, cudaStream_t st) {
     static int done[64] = {0};
     const int smem = da.L.total + 1024;
-    cudaError_t ce = set_smem_once(k_decode<kH, kRoute>, smem, done);
+    cudaError_t ce = set_smem_once(k_decode<kH, kMode>, smem, done);
     if (ce != cudaSuccess) return ce;
     const int G = num_sms_cached();
     if (G <= 0) return cudaErrorInvalidDevice;
     // every 16-row down tile needs a CTA, and every router row one of the CTAs' row slots
-    if (G < kH / 16 || (kRoute && G * kRouterRows < da.f.E)) return cudaErrorInvalidConfiguration;
+    if (G < kH / 16 || (kMode == kModeRoute && G * kRouterRows < da.f.E)) return cudaErrorInvalidConfiguration;
     // One CTA per SM.  CTAs read words other CTAs of the launch write, so they
     // must all be resident at once: a cooperative launch fails rather than
     // starting when they cannot be.
@@ -860,10 +934,10 @@ cudaError_t launch_dec_h(const DecArgs& da, const CUtensorMap& gu_map, const CUt
     attr[1].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, k_decode<kH, kRoute>, gu_map, gsb_map, dn_map, dsb_map, da);
+    return cudaLaunchKernelEx(&cfg, k_decode<kH, kMode>, gu_map, gsb_map, dn_map, dsb_map, da);
 }
 
-template <bool kRoute>
+template <int kMode>
 cudaError_t launch_dec(const DecArgs& da, cudaStream_t st) {
     CUtensorMap gu_map, gsb_map, dn_map, dsb_map;
     if (!make_gu_map(&gu_map, da.f) || !make_gsb_map(&gsb_map, da.f) || !make_dn_map(&dn_map, da.f))
@@ -874,9 +948,9 @@ cudaError_t launch_dec(const DecArgs& da, cudaStream_t st) {
         dsb_map = dn_map;   // not read
     }
     switch (da.f.H) {
-        case 512: return launch_dec_h<512, kRoute>(da, gu_map, gsb_map, dn_map, dsb_map, st);
-        case 1024: return launch_dec_h<1024, kRoute>(da, gu_map, gsb_map, dn_map, dsb_map, st);
-        case 2048: return launch_dec_h<2048, kRoute>(da, gu_map, gsb_map, dn_map, dsb_map, st);
+        case 512: return launch_dec_h<512, kMode>(da, gu_map, gsb_map, dn_map, dsb_map, st);
+        case 1024: return launch_dec_h<1024, kMode>(da, gu_map, gsb_map, dn_map, dsb_map, st);
+        case 2048: return launch_dec_h<2048, kMode>(da, gu_map, gsb_map, dn_map, dsb_map, st);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -926,15 +1000,33 @@ DecodeWs decode_ws_carve(uint8_t* base, int T, int E, int I, unsigned long long*
 
 cudaError_t launch_ffn_decode(const FfnArgs& a, const DecodeWs& w, cudaStream_t st) {
     DecArgs da = dec_args(a, w);
-    return launch_dec<false>(da, st);
+    return launch_dec<kModeTokens>(da, st);
 }
 
 bool decode_layer_supported(const FfnArgs& a) { return ffn_decode_supported(a) && a.E == 256; }
 
+bool ffn_rows_supported(const FfnArgs& a) {
+    if (!(a.mode == MOE_MODE_SCATTER && a.T >= 1 && a.K >= 1 && a.K <= 8 && a.G == 64 && a.E <= 256 &&
+          (a.H == 512 || a.H == 1024 || a.H == 2048) && a.I >= 128 && a.I <= 2048 && (a.I & (a.I - 1)) == 0))
+        return false;
+    const int G = num_sms_cached();
+    // a whole unit's four gate/up boxes fit in the ring beside the x slot of kMaxRows rows, and
+    // every CTA's units (at most all E experts' blocks) have room for their column tables
+    return G >= a.H / 16 && dec_layout(a.H, a.I, kMaxT).gu_slots >= 4 &&
+           (a.E * (a.I / kJ) + G - 1) / G <= row_units_cap(a.H);
+}
+
+cudaError_t launch_ffn_rows(const FfnArgs& a, cudaStream_t st) {
+    DecodeWs w = {};   // no launch counter, no logits: y_acc is not cleared, nothing is polled
+    DecArgs da = dec_args(a, w);
+    da.L = dec_layout(a.H, a.I, kMaxT);
+    return launch_dec<kModeRows>(da, st);
+}
+
 cudaError_t launch_decode_layer(const FfnArgs& a, const DecodeRoute& r, const DecodeWs& w, cudaStream_t st) {
     DecArgs da = dec_args(a, w);
     da.r = r;
-    return launch_dec<true>(da, st);
+    return launch_dec<kModeRoute>(da, st);
 }
 
 }  // namespace moe

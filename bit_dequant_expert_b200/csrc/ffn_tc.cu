@@ -88,6 +88,7 @@ struct TcArgs {
     int gateup;      // 1: gate/up + SwiGLU; 0: down + combine
     int nt;          // token rows per tile: kNTSplit (ksplit) or kNTWide
     int ksplit;      // 1: the K halves of every chunk on two MMA issuers
+    int skip_rows;   // experts of 1..skip_rows rows get no tiles (another launch takes them)
 };
 
 struct Tile {
@@ -101,7 +102,7 @@ __device__ __forceinline__ int tiles_per_block_row(const FfnArgs& a, int gateup)
 
 // Prefix of tiles per expert: pre[e] first tile of expert e, pre[E] first
 // shared tile, pre[E+1] total.  blockDim.x >= E.
-__device__ void tile_prefix(const FfnArgs& a, int gateup, int nt, int* pre, int* off) {
+__device__ void tile_prefix(const FfnArgs& a, int gateup, int nt, int skip_rows, int* pre, int* off) {
     __shared__ int warp_tot[32];
     const int MB = tiles_per_block_row(a, gateup);
     const int e = threadIdx.x;
@@ -112,7 +113,7 @@ __device__ void tile_prefix(const FfnArgs& a, int gateup, int nt, int* pre, int*
             set_error(a.err, MOE_ERR_BOUNDS);
             lo = hi = 0;
         }
-        tiles = (hi - lo + nt - 1) / nt * MB;
+        tiles = hi - lo <= skip_rows ? 0 : (hi - lo + nt - 1) / nt * MB;
         off[e] = lo;
         if (e == a.E - 1) off[a.E] = hi;
     }
@@ -235,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (size_t q = lo + tid; q < hi; q += kThreads)
             reinterpret_cast<float4*>(a.y_acc)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    tile_prefix(a, gateup, nt, sm.pre, sm.off);   // contains __syncthreads
+    tile_prefix(a, gateup, nt, ta.skip_rows, sm.pre, sm.off);   // contains __syncthreads
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     const int ntiles = sm.pre[a.E + 1];
@@ -677,7 +678,7 @@ bool ffn_tc_supported(const FfnArgs& a) {
            128 * (a.I / 64) * 4 <= kSbBytes;
 }
 
-cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
+cudaError_t launch_ffn_tc(const FfnArgs& a, int skip_rows, cudaStream_t st) {
     const int nmat = a.E + 1;
     CUtensorMap gu_map, d_map, x_map, h_map, x_map128, h_map128;
     if (!make_codes_map(&gu_map, a.gu_codes, nmat * 2 * a.I, a.H, 64)) return cudaErrorInvalidValue;
@@ -705,6 +706,7 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st) {
     // (a tcgen05.mma stream costs about the same per instruction for any N)
     ta.ksplit = (int64_t)a.T * a.K <= (int64_t)96 * a.E ? 1 : 0;
     ta.nt = ta.ksplit ? kNTSplit : kNTWide;
+    ta.skip_rows = skip_rows;
     k_ffn_tc<<<G, kThreads, smem, st>>>(gu_map, x_map, x_map128, gsb_map, ta);
     ce = cudaGetLastError();
     if (ce != cudaSuccess) return ce;

@@ -99,7 +99,8 @@ cudaError_t launch_router_logits(const RouterArgs& a, cudaStream_t st);
 size_t permute_ws_bytes(int T, int E, int K);
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t st);
 cudaError_t launch_ffn_simt(const FfnArgs& a, cudaStream_t st);
-cudaError_t launch_ffn_tc(const FfnArgs& a, cudaStream_t st);
+// Experts of 1..skip_rows rows get no tiles (0: every expert is computed).
+cudaError_t launch_ffn_tc(const FfnArgs& a, int skip_rows, cudaStream_t st);
 
 // Workspace sections of the decode kernels (T <= 8): the launch counter in
 // the workspace header and the tagged router logits (several copies).
@@ -113,6 +114,14 @@ DecodeWs decode_ws_carve(uint8_t* base, int T, int E, int I, unsigned long long*
 // Expert FFNs for T <= 8 (scatter mode): one launch, y_acc overwritten.
 bool ffn_decode_supported(const FfnArgs& a);
 cudaError_t launch_ffn_decode(const FfnArgs& a, const DecodeWs& w, cudaStream_t st);
+
+// The experts of 1..8 rows of a launch of any T (scatter mode), one unit per
+// (expert, 32 columns of I) as in the decode kernel, each MMA column a row of
+// the expert: x rows from xg (the gathered rows the tensor-core path reads),
+// w * y added into y_acc as it stands (the tensor-core launch with skip_rows 8
+// clears it and adds the other experts).
+bool ffn_rows_supported(const FfnArgs& a);
+cudaError_t launch_ffn_rows(const FfnArgs& a, cudaStream_t st);
 
 // The decode layer's router logits, top-k, permutation and expert FFNs in one
 // kernel (the routing outputs written as the route and permute calls would,

@@ -63,12 +63,23 @@ int32_t* err_word(void* ws) { return reinterpret_cast<int32_t*>(ws); }
 
 int32_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
+// The decode kernel's row-list launch takes the experts of at most 8 rows off
+// the tensor-core kernel.  Measured on one B200 (expert FFN, L2 flushed): at
+// H 2048 / I 512, T = 16 119 -> 107 us and T = 300 273 -> 261 us, but the
+// Zipf-skewed T = 512 layer 168 -> 175 us (its time is in the experts of many
+// rows) and T = 33 at H 512 42 -> 46 us (units too small to amortise the
+// per-unit handoffs).  So: the largest hidden size, at most 12 rows per expert
+// on average.
+bool split_small_experts(const FfnArgs& a) {
+    return a.H >= 2048 && ffn_rows_supported(a) && (int64_t)a.T * a.K <= (int64_t)12 * a.E;
+}
+
 // Implementation chosen for MOE_PATH_AUTO: the memory-bound decode kernel for
 // a handful of tokens, else the tensor-core kernel where its shape rules
 // hold, else the CUDA-core path.
 int32_t resolve_path(const FfnArgs& a) {
     if (ffn_decode_supported(a)) return MOE_PATH_GEMV;
-    if (ffn_tc_supported(a)) return MOE_PATH_TC;
+    if (ffn_tc_supported(a)) return split_small_experts(a) ? MOE_PATH_TC_GEMV : MOE_PATH_TC;
     return MOE_PATH_SIMT;
 }
 
@@ -241,7 +252,12 @@ int32_t moe_expert_ffn_path(const moe_config_t* cfg, int32_t T, const uint16_t* 
             return cuda_status(launch_ffn_decode(a, decode_ws(ws, cfg, T), s));
         case MOE_PATH_TC:
             if (!ffn_tc_supported(a)) return MOE_ERR_UNSUPPORTED;
-            return cuda_status(launch_ffn_tc(a, s));
+            return cuda_status(launch_ffn_tc(a, 0, s));
+        case MOE_PATH_TC_GEMV: {
+            if (!ffn_tc_supported(a) || !ffn_rows_supported(a)) return MOE_ERR_UNSUPPORTED;
+            const int32_t st = cuda_status(launch_ffn_tc(a, 8, s));
+            return st != MOE_OK ? st : cuda_status(launch_ffn_rows(a, s));
+        }
         default:
             return MOE_ERR_UNSUPPORTED;
     }
@@ -388,6 +404,7 @@ int32_t moe_launch_count(const moe_config_t* cfg, int32_t T, int32_t mode, int32
         case MOE_PATH_SIMT: ffn = 2; break;
         case MOE_PATH_GEMV: if (!ffn_decode_supported(a)) return -1; ffn = 1; break;
         case MOE_PATH_TC: if (!ffn_tc_supported(a)) return -1; ffn = 3; break;
+        case MOE_PATH_TC_GEMV: if (!ffn_tc_supported(a) || !ffn_rows_supported(a)) return -1; ffn = 4; break;
         default: return -1;
     }
     return route + permute + ffn + 1;

@@ -95,6 +95,10 @@ typedef struct {
 #define MOE_PATH_SIMT 1    /* CUDA-core dequant + dot products, any T */
 #define MOE_PATH_GEMV 2    /* memory-bound split-K GEMV, few rows per expert */
 #define MOE_PATH_TC 3      /* TMA; dequant in registers into tensor memory (A); tcgen05 MMA */
+#define MOE_PATH_TC_GEMV 4 /* scatter mode: MOE_PATH_TC for experts of more than 8 rows, then
+                             the split-K GEMV kernel over the rows of the others (T unrestricted);
+                             MOE_PATH_AUTO takes it when hidden >= 2048 and
+                             T * top_k <= 12 * num_experts */
 
 /* Bytes of workspace that the calls need for up to max_tokens tokens; 0 if
  * the configuration is unsupported.  Caller allocates it (256-byte aligned)
