@@ -88,7 +88,6 @@ struct TcArgs {
     int gateup;      // 1: gate/up + SwiGLU; 0: down + combine
     int nt;          // token rows per tile: kNTSplit (ksplit) or kNTWide
     int ksplit;      // 1: the K halves of every chunk on two MMA issuers
-    int skip_rows;   // experts of 1..skip_rows rows get no tiles (another launch takes them)
 };
 
 struct Tile {
@@ -101,8 +100,10 @@ __device__ __forceinline__ int tiles_per_block_row(const FfnArgs& a, int gateup)
 }
 
 // Prefix of tiles per expert: pre[e] first tile of expert e, pre[E] first
-// shared tile, pre[E+1] total.  blockDim.x >= E.
-__device__ void tile_prefix(const FfnArgs& a, int gateup, int nt, int skip_rows, int* pre, int* off) {
+// shared tile, pre[E+1] total.  blockDim.x >= E.  Experts of 1..kSkipRows
+// rows get no tiles (another launch takes them).
+template <int kSkipRows>
+__device__ void tile_prefix(const FfnArgs& a, int gateup, int nt, int* pre, int* off) {
     __shared__ int warp_tot[32];
     const int MB = tiles_per_block_row(a, gateup);
     const int e = threadIdx.x;
@@ -113,7 +114,8 @@ __device__ void tile_prefix(const FfnArgs& a, int gateup, int nt, int skip_rows,
             set_error(a.err, MOE_ERR_BOUNDS);
             lo = hi = 0;
         }
-        tiles = hi - lo <= skip_rows ? 0 : (hi - lo + nt - 1) / nt * MB;
+        tiles = (hi - lo + nt - 1) / nt * MB;
+        if (kSkipRows > 0 && hi - lo <= kSkipRows) tiles = 0;
         off[e] = lo;
         if (e == a.E - 1) off[a.E] = hi;
     }
@@ -175,6 +177,7 @@ __device__ __forceinline__ int wrow_gate(const FfnArgs& a, const Tile& tl) { ret
 __device__ __forceinline__ int wrow_up(const FfnArgs& a, const Tile& tl) { return tl.e * 2 * a.I + a.I + 64 * tl.mb; }
 __device__ __forceinline__ int wrow_down(const FfnArgs& a, const Tile& tl) { return tl.e * a.H + 128 * tl.mb; }
 
+template <int kSkipRows>
 __global__ void __launch_bounds__(kThreads, 1)
     k_ffn_tc(const __grid_constant__ CUtensorMap codes_map, const __grid_constant__ CUtensorMap b_map64,
              const __grid_constant__ CUtensorMap b_map128, const __grid_constant__ CUtensorMap sb_map,
@@ -236,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (size_t q = lo + tid; q < hi; q += kThreads)
             reinterpret_cast<float4*>(a.y_acc)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    tile_prefix(a, gateup, nt, ta.skip_rows, sm.pre, sm.off);   // contains __syncthreads
+    tile_prefix<kSkipRows>(a, gateup, nt, sm.pre, sm.off);   // contains __syncthreads
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     const int ntiles = sm.pre[a.E + 1];
@@ -695,7 +698,11 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, int skip_rows, cudaStream_t st) {
     k_gather_rows<<<(grows + 7) / 8, 256, 0, st>>>(a);
     const int smem = (int)sizeof(Smem) + 1024;
     static int done[64] = {0};
-    cudaError_t ce = set_smem_once(k_ffn_tc, smem, done);
+    // experts of at most 8 rows left to the decode kernel's row-list launch, or none
+    auto kern = skip_rows == 8 ? k_ffn_tc<8> : k_ffn_tc<0>;
+    if (skip_rows != 0 && skip_rows != 8) return cudaErrorInvalidValue;
+    static int done8[64] = {0};
+    cudaError_t ce = set_smem_once(kern, smem, skip_rows == 8 ? done8 : done);
     if (ce != cudaSuccess) return ce;
     const int G = num_sms();
     if (G <= 0) return cudaErrorInvalidDevice;
@@ -706,12 +713,11 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, int skip_rows, cudaStream_t st) {
     // (a tcgen05.mma stream costs about the same per instruction for any N)
     ta.ksplit = (int64_t)a.T * a.K <= (int64_t)96 * a.E ? 1 : 0;
     ta.nt = ta.ksplit ? kNTSplit : kNTWide;
-    ta.skip_rows = skip_rows;
-    k_ffn_tc<<<G, kThreads, smem, st>>>(gu_map, x_map, x_map128, gsb_map, ta);
+    kern<<<G, kThreads, smem, st>>>(gu_map, x_map, x_map128, gsb_map, ta);
     ce = cudaGetLastError();
     if (ce != cudaSuccess) return ce;
     ta.gateup = 0;
-    k_ffn_tc<<<G, kThreads, smem, st>>>(d_map, h_map, h_map128, dsb_map, ta);
+    kern<<<G, kThreads, smem, st>>>(d_map, h_map, h_map128, dsb_map, ta);
     return cudaGetLastError();
 }
 
