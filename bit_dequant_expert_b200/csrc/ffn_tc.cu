@@ -656,17 +656,28 @@ __global__ void __launch_bounds__(256) k_gather_rows(FfnArgs a) {
         tok = (p >= 0 && p < a.T * a.K) ? p / a.K : 0;
         if (p < 0 || p >= a.T * a.K) set_error(a.err, MOE_ERR_BOUNDS);
     }
-    const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)tok * a.H);
-    uint4* dst = reinterpret_cast<uint4*>(a.xg + (size_t)row * a.H);
-    // each 8 inputs in the split order (0,4,1,5,2,6,3,7) of the dequantised weights
-    for (int c = lane; c < a.H / 8; c += 32) {
-        const uint4 v = src[c];
-        uint4 r;
-        r.x = prmt(v.x, v.z, 0x5410);
-        r.y = prmt(v.x, v.z, 0x7632);
-        r.z = prmt(v.y, v.w, 0x5410);
-        r.w = prmt(v.y, v.w, 0x7632);
-        dst[c] = r;
+    const uint4* __restrict__ src = reinterpret_cast<const uint4*>(a.x + (size_t)tok * a.H);
+    uint4* __restrict__ dst = reinterpret_cast<uint4*>(a.xg + (size_t)row * a.H);
+    // each 8 inputs in the split order (0,4,1,5,2,6,3,7) of the dequantised weights; a lane
+    // issues up to kPer loads before its stores (one round covers H = 2048)
+    constexpr int kPer = 8;
+    const int n8 = a.H / 8;
+    for (int c0 = lane; c0 < n8; c0 += 32 * kPer) {
+        uint4 v[kPer];
+#pragma unroll
+        for (int i = 0; i < kPer; ++i)
+            if (c0 + 32 * i < n8) v[i] = __ldg(src + c0 + 32 * i);
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            if (c0 + 32 * i < n8) {
+                uint4 r;
+                r.x = prmt(v[i].x, v[i].z, 0x5410);
+                r.y = prmt(v[i].x, v[i].z, 0x7632);
+                r.z = prmt(v[i].y, v[i].w, 0x5410);
+                r.w = prmt(v[i].y, v[i].w, 0x7632);
+                dst[c0 + 32 * i] = r;
+            }
+        }
     }
 }
 
