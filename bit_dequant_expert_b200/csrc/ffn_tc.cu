@@ -67,6 +67,7 @@ static_assert(2 * kNTWide <= kACol0, "TMEM budget");
 constexpr int kAStageCols = kBK / 2;     // bf16 pairs per 32-bit column
 constexpr int kTmemCols = 512;
 constexpr int kTabs = 4;                 // column tables in flight (down epilogue)
+constexpr int kStageStride = 36;         // floats per staged column (32 rows + 4: conflict-free float4 reads)
 constexpr int kSbBytes = 16384;          // one tile's (scale, bias) words: 128 rows x up to 32 groups
 static_assert(kACol0 + kStages * kAStageCols <= kTmemCols, "TMEM budget");
 
@@ -80,8 +81,10 @@ struct Smem {
     float w[kTabs][kNTWide];
     int pre[260];
     int off[260];                                // offsets[0..E], cached
+    float stage[4][16 * kStageStride];           // scatter epilogue: a warp's 16 columns x 32 rows
     uint32_t tmem_base;
 };
+static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory per block");
 
 struct TcArgs {
     FfnArgs f;
@@ -541,15 +544,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                             *reinterpret_cast<uint32_t*>(dst + (size_t)(tl.r0 + col) * a.H + (n & ~1)) = pk;
                     }
                 } else {
-                    // fp32 y_acc: w * y added into the token's row
-                    const int n = 128 * tl.mb + 32 * q + lane;
+                    // fp32 y_acc: w * y added into the token's row.  The warp's 32 rows x 16
+                    // columns go through shared memory so that each lane adds 4 consecutive
+                    // outputs of one token with one vector reduction
+                    float* stg = sm.stage[q];
+                    const int n0 = 128 * tl.mb + 32 * q;
 #pragma unroll
-                    for (int c = 0; c < 16; ++c) {
+                    for (int c = 0; c < 16; ++c) stg[c * kStageStride + lane] = sm.w[slot][c0 + c] * __uint_as_float(v[c]);
+                    __syncwarp();
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int c = (lane >> 3) + 4 * i, r4 = lane & 7;   // column, row quad
                         const int col = c0 + c;
-                        if (col < tl.nr)
-                            atomicAdd(a.y_acc + (size_t)sm.tok[slot][col] * a.H + n,
-                                      sm.w[slot][col] * __uint_as_float(v[c]));
+                        if (col < tl.nr) {
+                            const float4 f = *reinterpret_cast<const float4*>(stg + c * kStageStride + 4 * r4);
+                            red_add_v4(a.y_acc + (size_t)sm.tok[slot][col] * a.H + n0 + 4 * r4, f.x, f.y, f.z, f.w);
+                        }
                     }
+                    __syncwarp();   // the next chunk overwrites the staging area
                 }
             }
             if (!gateup) {
