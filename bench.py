@@ -366,7 +366,7 @@ def run_decode(device, steps, warmup, world, peaks):
     roofline_ffn = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": achieved / peaks["hbm_gbs"],
                     "traffic": profiled_traffic("ffn_decode", "ffn_decode_t1_ncu.txt"),
-                    "kernel": "k_decode<false> (moe_expert_ffn at T=1: gate/up + SwiGLU, then down + vector reductions into y_acc)",
+                    "kernel": "k_decode<0> (moe_expert_ffn at T=1: gate/up + SwiGLU, then down + vector reductions into y_acc)",
                     "algorithmic_bytes": FFN_BYTES_T1, "avg_launch_us": ffn_ms * 1e3,
                     "peak_source": peaks["source"] + " hbm_gbs"}
 
@@ -395,7 +395,7 @@ def run_decode(device, steps, warmup, world, peaks):
     roofline = {"bound": "hbm", "achieved": layer_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": layer_gbs / peaks["hbm_gbs"],
                 "traffic": profiled_traffic("ffn_decode", "decode_layer_t1_ncu.txt"),
-                "kernel": "moe_decode_layer: k_decode<true> (route + permute + expert FFN) + k_combine_scatter",
+                "kernel": "moe_decode_layer: k_decode<1> (route + permute + expert FFN) + k_combine_scatter",
                 "algorithmic_bytes": layer_bytes, "avg_layer_us": layer_us, "launches_per_layer": 2,
                 "traffic_note": "ncu DRAM bytes of the layer kernel's launch",
                 "peak_source": peaks["source"] + " hbm_gbs"}
