@@ -19,7 +19,13 @@
 //    into y_acc with vector reductions.  At T = 1 the 9 experts x 16 blocks are
 //    one unit on each of 144 SMs.  Every unit computes all T tokens (the
 //    MMA's N = 8 columns); a token's routing weight is zero where it did not
-//    pick the expert.
+//    pick the expert.  Each warp stages its 16-row down tiles in shared memory
+//    so that one vector reduction adds 4 consecutive rows of one token.
+//  - Three modes: the T <= 8 tokens of a launch (expert FFN call), the same
+//    with routing fused in (decode layer), and a row list (any T): units of
+//    the experts that hold 1..8 rows, whose MMA columns are those rows, x rows
+//    brought per unit from the gathered rows, the tensor-core kernel taking
+//    every other expert.
 //  - Group-factored dequantisation: w = s q + b over a group of inputs is
 //    s (128 + q) + (b - 128 s), so the MMAs run on the exact bf16 values
 //    128 + q (one mask-and-or per two weights) and each group's fp32 partial
