@@ -13,7 +13,7 @@ from gpu_util import check_output, check_permutation_props, check_routing, run_l
 pytestmark = pytest.mark.gpu
 
 SCATTER, PAIRS = 0, 1
-AUTO, SIMT, GEMV, TC = 0, 1, 2, 3
+AUTO, SIMT, GEMV, TC, TC_GEMV = 0, 1, 2, 3, 4
 
 
 def _decode_shape(T):
@@ -53,12 +53,13 @@ def test_decode_shape_past_the_crossover():
 
 @pytest.mark.parametrize("path,mode,T", [(AUTO, SCATTER, 1), (AUTO, SCATTER, 6), (GEMV, SCATTER, 3),
                                          (SIMT, SCATTER, 8), (SIMT, PAIRS, 8), (TC, SCATTER, 33),
-                                         (TC, PAIRS, 33)])
+                                         (TC, PAIRS, 33), (TC_GEMV, SCATTER, 33), (TC_GEMV, SCATTER, 300)])
 def test_without_shared_expert(path, mode, T):
     """has_shared = 0: only the routed experts contribute; the matrices at
     index E are never read.  Checked against the oracle without the shared
     expert, with the shared expert's codes set to values that would show if
-    they were read."""
+    they were read.  The split path at T = 33 leaves the tensor-core kernel
+    no tile at all (every expert holds at most 8 rows)."""
     from bit_dequant_expert_b200.layer import MoELayer
     lay = dict(gen.make_layer(gen.config(0).with_T(T), 1))
     for name in ("gu_codes", "d_codes"):
