@@ -638,30 +638,50 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tab.sel[warp * 8 + lane] = e_sel;
                     tab.selw[warp * 8 + lane] = w_sel;
                 }
-            }
-            named_barrier(1, kWarps * 32);
-            // ---- active experts: the shared one, then the selected ones by index
-            if (tid < T * 8) atomicOr(&tab.bitmap[tab.sel[tid] >> 5], 1u << (tab.sel[tid] & 31));
-            named_barrier(1, kWarps * 32);
-            if (tid < E) {
-                const int wdx = tid >> 5;
-                int below = __popc(tab.bitmap[wdx] & ((1u << (tid & 31)) - 1u));
-                for (int q = 0; q < wdx; ++q) below += __popc(tab.bitmap[q]);
-                if ((tab.bitmap[wdx] >> (tid & 31)) & 1u) {
-                    tab.slot_e[first + below] = tid;
-                    tab.slot_of[tid] = first + below;
+                if (T == 1) {
+                    // one token: its 8 (distinct) experts ranked by index are the routed slots
+                    int rank = 0;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) rank += __shfl_sync(0xFFFFFFFFu, e_sel, j) < e_sel ? 1 : 0;
+                    if (lane < 8) {
+                        tab.slot_e[first + rank] = e_sel;
+                        tab.slot_of[e_sel] = first + rank;
+                        tab.wsel[first + rank][0] = w_sel;
+                    }
+                    if (lane == 0) {
+                        tab.A = first + 8;
+                        if (sh) tab.slot_e[0] = E;
+                    }
                 }
             }
-            if (tid == 0) {
-                int tot = 0;
-                for (int q = 0; q < 8; ++q) tot += __popc(tab.bitmap[q]);
-                tab.A = first + tot;
-                if (sh) tab.slot_e[0] = E;
+            if (T == 1) {
+                named_barrier(1, kWarps * 32);           // the active list and its weights
+                if (tid == 0) mbar_arrive(list_ready);   // are ready for the producer
+            } else {
+                named_barrier(1, kWarps * 32);
+                // ---- active experts: the shared one, then the selected ones by index
+                if (tid < T * 8) atomicOr(&tab.bitmap[tab.sel[tid] >> 5], 1u << (tab.sel[tid] & 31));
+                named_barrier(1, kWarps * 32);
+                if (tid < E) {
+                    const int wdx = tid >> 5;
+                    int below = __popc(tab.bitmap[wdx] & ((1u << (tid & 31)) - 1u));
+                    for (int q = 0; q < wdx; ++q) below += __popc(tab.bitmap[q]);
+                    if ((tab.bitmap[wdx] >> (tid & 31)) & 1u) {
+                        tab.slot_e[first + below] = tid;
+                        tab.slot_of[tid] = first + below;
+                    }
+                }
+                if (tid == 0) {
+                    int tot = 0;
+                    for (int q = 0; q < 8; ++q) tot += __popc(tab.bitmap[q]);
+                    tab.A = first + tot;
+                    if (sh) tab.slot_e[0] = E;
+                }
+                named_barrier(1, kWarps * 32);
+                if (tid == 0) mbar_arrive(list_ready);   // the active list is ready for the producer
+                if (tid < T * 8) tab.wsel[tab.slot_of[tab.sel[tid]]][tid >> 3] = tab.selw[tid];
+                named_barrier(1, kWarps * 32);           // and the weights for every compute warp
             }
-            named_barrier(1, kWarps * 32);
-            if (tid == 0) mbar_arrive(list_ready);   // the active list is ready for the producer
-            if (tid < T * 8) tab.wsel[tab.slot_of[tab.sel[tid]]][tid >> 3] = tab.selw[tid];
-            named_barrier(1, kWarps * 32);           // and the weights for every compute warp
             // ---- the routing outputs, by the last CTA (the four calls' results)
             if (b == G - 1) {
                 const int np = T * 8;
