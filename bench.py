@@ -717,8 +717,10 @@ def run_ncu_case(case, device, calls):
     from bit_dequant_expert_b200 import MOE_MODE_PAIRS, MOE_MODE_SCATTER
     from bit_dequant_expert_b200.layer import MoELayer, to_device
     prefill = case.startswith("prefill")
-    spec = gen.config(3 if prefill else 1)
-    lay = gen.make_layer(spec, 0)
+    # split-t16: 16 tokens of the decode layer shape through the split path (the tensor-core
+    # kernel for the shared expert, the decode kernel's row-list launch for the others)
+    spec = gen.config(3) if prefill else gen.config(1).with_T(16) if case == "split-t16" else gen.config(1)
+    lay = gen.make_layer(spec, 3 if case == "split-t16" else 0)
     T = spec.T
     L = MoELayer(lay, max_tokens=T, device=device,
                  mode=MOE_MODE_PAIRS if prefill else MOE_MODE_SCATTER)
@@ -794,7 +796,7 @@ def main(argv=None):
     ap.add_argument("--prefill-only", action="store_true",
                     help="measure only the T=2048 prefill layer (its line replaces the decode line)")
     ap.add_argument("--ncu-case", choices=("decode-ffn", "decode-layer", "prefill-ffn", "prefill-layer", "gdn-decode",
-                                                   "gdn-prefill"),
+                                                   "gdn-prefill", "split-t16"),
                     help="a small case for a profiler capture: one synthetic layer, route + permute, then "
                          "--steps calls of the named kernel (decode: config 1 layer 0, T=1; prefill: "
                          "config 3, T=2048); prints the device error word and nothing timed")
